@@ -1,0 +1,94 @@
+"""Seeded synthetic inputs shared by the tests, the bench and the oracle checks.
+
+This module only names workload shapes and draws random numbers; it holds none
+of the attention arithmetic, so both the CUDA path's callers and the oracle
+checks may use it without sharing any of the method.
+
+Recipe: one CPU ``torch.Generator`` per tensor, seeded ``seed``, ``seed + 1``,
+``seed + 2`` for q, k, v; ``randn`` in float32 (iid N(0, 1)), then rounded to
+bfloat16 on the host. The identical bf16 tensors go to the GPU and, upcast
+exactly, to the oracle.
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import torch
+
+SEED_Q = 1234
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    Nq: int
+    Nk: int
+    d: int
+    causal: bool = True
+    window_left: int = -1
+    decode: bool = False          # single-query decode over a contiguous KV cache
+    fp32_out: bool = False
+    note: str = field(default="", compare=False)
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / (self.d ** 0.5)
+
+
+# The five workloads the pages' scenarios translate into (tiny exact check,
+# MHA causal prefill at 2K and 8K, GQA sliding window at 32K, GQA decode).
+TINY = Workload("tiny exact attention B1 H2 N128 d64", 1, 2, 2, 128, 128, 64,
+                causal=False, fp32_out=True)
+TINY_CAUSAL = Workload("tiny exact attention B1 H2 N128 d64 causal", 1, 2, 2, 128, 128, 64,
+                       causal=True, fp32_out=True)
+MHA_2K = Workload("MHA causal prefill B4 H32 N2048 d128", 4, 32, 32, 2048, 2048, 128)
+MHA_8K = Workload("MHA causal prefill B4 H32 N8192 d128", 4, 32, 32, 8192, 8192, 128)
+GQA_SWA_32K = Workload("GQA sliding-window prefill B1 N32768 Hq32 Hkv8 d128 window_left4096",
+                       1, 32, 8, 32768, 32768, 128, causal=True, window_left=4096)
+GQA_DECODE = Workload("GQA decode B64 L8192 Hq32 Hkv8 d128", 64, 32, 8, 1, 8192, 128,
+                      causal=True, decode=True)
+
+ALL = [TINY, TINY_CAUSAL, MHA_2K, MHA_8K, GQA_SWA_32K, GQA_DECODE]
+
+
+def _randn(shape, seed: int) -> torch.Tensor:
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    return torch.randn(*shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
+
+
+def make_qkv(B, Hq, Hkv, Nq, Nk, d, seed: int = SEED_Q):
+    """bf16 CPU tensors q ``[B,Nq,Hq,d]``, k and v ``[B,Nk,Hkv,d]``."""
+    q = _randn((B, Nq, Hq, d), seed)
+    k = _randn((B, Nk, Hkv, d), seed + 1)
+    v = _randn((B, Nk, Hkv, d), seed + 2)
+    return q, k, v
+
+
+def make_decode(B, Hq, Hkv, Lmax, d, seed: int = SEED_Q):
+    """bf16 CPU tensors q ``[B,Hq,d]``, k_cache and v_cache ``[B,Lmax,Hkv,d]``."""
+    q = _randn((B, Hq, d), seed)
+    k = _randn((B, Lmax, Hkv, d), seed + 1)
+    v = _randn((B, Lmax, Hkv, d), seed + 2)
+    return q, k, v
+
+
+def make_for(w: Workload, seed: int = SEED_Q):
+    if w.decode:
+        return make_decode(w.B, w.Hq, w.Hkv, w.Nk, w.d, seed)
+    return make_qkv(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, seed)
+
+
+def ragged_seqlens(B: int, Lmax: int, seed: int = SEED_Q + 7) -> torch.Tensor:
+    """int32 ``[B]`` cache lengths in ``[1, Lmax]`` (a mix of short and full rows)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    s = torch.randint(1, Lmax + 1, (B,), generator=g, dtype=torch.int32)
+    s[0] = Lmax
+    if B > 1:
+        s[1] = 1
+    return s

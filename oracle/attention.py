@@ -1,0 +1,324 @@
+"""fp64 CPU oracle for exact scaled-dot-product attention (test infrastructure).
+
+This module is the *definition* the CUDA kernels are checked against. It is
+used only by the tests, by ``__graft_entry__.smoke()`` and by the CPU-baseline
+leg of ``bench.py``; the product path never imports it.
+
+Sources (page title, then section):
+
+* "Attention Is O(n²): FlashAttention vs Linear Attention", section
+  "Why Attention Is O(n²)": the plain operation ``softmax(Q Kᵀ / sqrt(d)) V``;
+  section "Wall-Clock Impact of Tiling": the naive reference that materialises
+  the full score matrix, and the tiled online-softmax loop (section
+  "FlashAttention — Same FLOPs, Linear Memory") that reaches the same result.
+* "Modern Attention: MQA, GQA, FlashAttention, Sliding Window and RoPE",
+  section 3 "FlashAttention: exact, but IO-aware" (running max / running
+  denominator, worked example on scores [1, 3]) and section 4
+  "Sliding-window attention" (the n = 8, W = 3 mask).
+* "Chapter 3: MHA Limitations, MQA, GQA, and FlashAttention", section 3.3
+  (query head i reads K/V group i // (H // G)) and section 3.5 (merging two
+  partial softmax states by rescaling to the common maximum).
+
+Readings taken where the pages are silent or garbled (all listed in the
+design notes):
+
+* ``window_left`` counts the keys strictly before the query's own position,
+  so the page's "last W tokens" is ``window_left = W - 1``.
+* Causal alignment for ``Nq != Nk`` is bottom-right: query row i sits at key
+  position ``qpos(i) = i + Nk - Nq``.
+* A window without ``causal`` limits the left side only.
+* A row with no allowed key has O = 0 and LSE = -inf.
+* LSE is the natural log-sum-exp of the *scaled* scores.
+* The merge rule lost from section 3.5 is restated as
+  ``m' = max(m_a, m_b)``, ``l' = l_a e^(m_a-m') + l_b e^(m_b-m')``,
+  ``acc' = acc_a e^(m_a-m') + acc_b e^(m_b-m')``.
+
+Layouts: Q ``[B, Nq, Hq, d]``, K/V ``[B, Nk, Hkv, d]``, O ``[B, Nq, Hq, d]``,
+LSE ``[B, Hq, Nq]``.  Inputs may be any real dtype; they are upcast exactly to
+float64 before any arithmetic.
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+NEG_INF = -np.inf
+
+
+def _f64(x) -> np.ndarray:
+    """Exact upcast to float64 (bf16/fp16/fp32 values are all representable)."""
+    if hasattr(x, "detach"):  # a torch tensor: go through float32 (exact for bf16)
+        x = x.detach().to("cpu").float().numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def allowed_mask(Nq: int, Nk: int, causal: bool, window_left: int) -> np.ndarray:
+    """Boolean ``[Nq, Nk]`` mask of the (query, key) pairs that take part.
+
+    Query row ``i`` sits at key position ``qpos = i + Nk - Nq`` (bottom-right
+    alignment). Key ``j`` is allowed when ``j <= qpos`` (if ``causal``) and
+    ``j >= qpos - window_left`` (if ``window_left >= 0``). With ``Nq = Nk = 8``,
+    ``causal`` and ``window_left = 2`` this is the "last W = 3 tokens" diagram
+    of "Modern Attention ...", section 4 "Sliding-window attention".
+    """
+    i = np.arange(Nq)[:, None]
+    j = np.arange(Nk)[None, :]
+    qpos = i + (Nk - Nq)
+    ok = np.ones((Nq, Nk), dtype=bool)
+    if causal:
+        ok &= j <= qpos
+    if window_left is not None and window_left >= 0:
+        ok &= j >= qpos - window_left
+    return ok
+
+
+def _head_attention(qh, kh, vh, scale, mask):
+    """One (batch, query head): materialise S and P, return (O, LSE, P).
+
+    Steps follow the plain definition ("Attention Is O(n²) ...", section
+    "Why Attention Is O(n²)"): S = scale * Q Kᵀ; masked entries -> -inf;
+    P = softmax over each row (max-subtracted, as in the naive reference of
+    section "Wall-Clock Impact of Tiling"); O = P V; LSE = m + ln(sum exp(S - m)).
+    """
+    S = scale * (qh @ kh.T)                       # [rows, Nk]
+    S = np.where(mask, S, NEG_INF)
+    m = S.max(axis=1)                             # -inf for a row with no key
+    has_key = np.isfinite(m)
+    m_safe = np.where(has_key, m, 0.0)
+    E = np.exp(S - m_safe[:, None])               # exp(-inf) = 0 for masked keys
+    l = E.sum(axis=1)
+    P = np.zeros_like(E)
+    P[has_key] = E[has_key] / l[has_key, None]
+    O = P @ vh
+    lse = np.full(m.shape, NEG_INF)
+    lse[has_key] = m[has_key] + np.log(l[has_key])
+    return O, lse, P
+
+
+def oracle_attention(q, k, v, causal: bool = False, window_left: int = -1,
+                     scale: float | None = None, row_block: int = 512):
+    """Exact attention in float64. Returns ``(O [B,Nq,Hq,d], LSE [B,Hq,Nq])``.
+
+    Query head ``hq`` reads K/V head ``hq // (Hq // Hkv)`` ("Chapter 3 ...",
+    section 3.3: each K/V group is repeated H // G times). S and P are
+    materialised for blocks of ``row_block`` query rows against all ``Nk`` keys.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Nq, Hq, d = q.shape
+    Bk, Nk, Hkv, dk = k.shape
+    assert Bk == B and dk == d and v.shape == k.shape
+    assert Hq % Hkv == 0, "query heads must be a multiple of K/V heads"
+    group = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    mask = allowed_mask(Nq, Nk, causal, window_left)
+    O = np.zeros((B, Nq, Hq, d))
+    LSE = np.full((B, Hq, Nq), NEG_INF)
+    for b in range(B):
+        for hq in range(Hq):
+            hk = hq // group
+            for r0 in range(0, Nq, row_block):
+                r1 = min(r0 + row_block, Nq)
+                o, lse, _ = _head_attention(q[b, r0:r1, hq], k[b, :, hk], v[b, :, hk],
+                                            scale, mask[r0:r1])
+                O[b, r0:r1, hq] = o
+                LSE[b, hq, r0:r1] = lse
+    return O, LSE
+
+
+def oracle_attention_rows(q, k, v, b: int, hq: int, rows, causal: bool = False,
+                          window_left: int = -1, scale: float | None = None):
+    """Selected query rows of one (batch, head): ``(O [len(rows), d], LSE [len(rows)])``.
+
+    Same arithmetic as :func:`oracle_attention`, evaluated only for the listed
+    rows so that full-size problems can be checked on sampled outputs.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Nq, Hq, d = q.shape
+    _, Nk, Hkv, _ = k.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    rows = np.asarray(rows, dtype=np.int64)
+    hk = hq // (Hq // Hkv)
+    mask = allowed_mask(Nq, Nk, causal, window_left)[rows]
+    o, lse, _ = _head_attention(q[b, rows, hq], k[b, :, hk], v[b, :, hk], scale, mask)
+    return o, lse
+
+
+def oracle_probabilities(q, k, causal=False, window_left=-1, scale=None, b=0, hq=0):
+    """The full probability matrix P ``[Nq, Nk]`` of one (batch, head) (small cases)."""
+    q, k = _f64(q), _f64(k)
+    _, Nq, Hq, d = q.shape
+    _, Nk, Hkv, _ = k.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    hk = hq // (Hq // Hkv)
+    mask = allowed_mask(Nq, Nk, causal, window_left)
+    _, _, P = _head_attention(q[b, :, hq], k[b, :, hk], np.zeros((Nk, 1)), scale, mask)
+    return P
+
+
+def oracle_decode(q, k_cache, v_cache, seqlens=None, window_left: int = -1,
+                  scale: float | None = None):
+    """Single-query decode over a contiguous KV cache.
+
+    ``q [B, Hq, d]``, ``k_cache/v_cache [B, Lmax, Hkv, d]``, ``seqlens [B]``
+    (None: all ``Lmax``). The new query's own K/V are already in the cache
+    ("Chapter 3 ...", section 3.1: a new token's K/V are appended before it
+    attends), so it sits at position ``seqlen - 1`` and sees keys
+    ``[max(0, seqlen-1-window_left), seqlen)``. This is exactly the last row of
+    causal prefill with ``Nq = 1`` and ``Nk = seqlen``.
+    Returns ``(O [B, Hq, d], LSE [B, Hq])``.
+    """
+    q, kc, vc = _f64(q), _f64(k_cache), _f64(v_cache)
+    B, Hq, d = q.shape
+    _, Lmax, Hkv, _ = kc.shape
+    if seqlens is None:
+        seqlens = [Lmax] * B
+    seqlens = [int(s) for s in np.asarray(seqlens).reshape(-1)]
+    O = np.zeros((B, Hq, d))
+    LSE = np.full((B, Hq), NEG_INF)
+    for b in range(B):
+        L = seqlens[b]
+        if L <= 0:
+            continue
+        o, lse = oracle_attention(q[b:b + 1, None], kc[b:b + 1, :L], vc[b:b + 1, :L],
+                                  causal=True, window_left=window_left, scale=scale)
+        O[b] = o[0, 0]
+        LSE[b] = lse[0, :, 0]
+    return O, LSE
+
+
+# ---------------------------------------------------------------------------
+# Second, independent formulations used only to check the one above.
+# ---------------------------------------------------------------------------
+
+def online_softmax(xs):
+    """Softmax of a 1-D list in one pass with a running max and denominator.
+
+    "Modern Attention ...", section 3: when a new value raises the maximum, the
+    running denominator is rescaled by exp(old_max - new_max). Returns
+    ``(probabilities, final_max, denominator)``.
+    """
+    m, den = -math.inf, 0.0
+    for x in xs:
+        new_m = max(m, x)
+        den = (den * math.exp(m - new_m) if den else 0.0) + math.exp(x - new_m)
+        m = new_m
+    return [math.exp(x - m) / den for x in xs], m, den
+
+
+def tiled_attention(q, k, v, causal=False, window_left=-1, scale=None,
+                    block_q: int = 32, block_k: int = 32):
+    """The tiled loop with running max / running sum / rescaled accumulator.
+
+    "Attention Is O(n²) ...", section "FlashAttention — Same FLOPs, Linear
+    Memory": outer loop over query blocks, inner loop over key/value blocks;
+    the accumulator and running sum are rescaled by exp(old_max - new_max) and
+    the output is divided by the running sum at the end. Masked scores are
+    -inf (they contribute exp(-inf) = 0). fp64 throughout.
+    Returns ``(O [B,Nq,Hq,d], LSE [B,Hq,Nq])``.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Nq, Hq, d = q.shape
+    _, Nk, Hkv, _ = k.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    group = Hq // Hkv
+    mask = allowed_mask(Nq, Nk, causal, window_left)
+    O = np.zeros((B, Nq, Hq, d))
+    LSE = np.full((B, Hq, Nq), NEG_INF)
+    for b in range(B):
+        for hq in range(Hq):
+            hk = hq // group
+            for i0 in range(0, Nq, block_q):
+                i1 = min(i0 + block_q, Nq)
+                Qi = q[b, i0:i1, hq]
+                acc = np.zeros((i1 - i0, d))
+                run_max = np.full(i1 - i0, -np.inf)
+                run_sum = np.zeros(i1 - i0)
+                for j0 in range(0, Nk, block_k):
+                    j1 = min(j0 + block_k, Nk)
+                    Sij = scale * (Qi @ k[b, j0:j1, hk].T)
+                    Sij = np.where(mask[i0:i1, j0:j1], Sij, -np.inf)
+                    new_max = np.maximum(run_max, Sij.max(axis=1))
+                    safe = np.where(np.isfinite(new_max), new_max, 0.0)
+                    Pij = np.exp(Sij - safe[:, None])
+                    corr = np.exp(run_max - safe)
+                    acc = acc * corr[:, None] + Pij @ v[b, j0:j1, hk]
+                    run_sum = run_sum * corr + Pij.sum(axis=1)
+                    run_max = new_max
+                ok = run_sum > 0
+                out = np.zeros_like(acc)
+                out[ok] = acc[ok] / run_sum[ok, None]
+                O[b, i0:i1, hq] = out
+                lse = np.full(i1 - i0, -np.inf)
+                lse[ok] = run_max[ok] + np.log(run_sum[ok])
+                LSE[b, hq, i0:i1] = lse
+    return O, LSE
+
+
+def merge_partials(parts):
+    """Merge partial softmax states ``[(m, l, acc), ...]`` of disjoint key sets.
+
+    "Chapter 3 ...", section 3.5: the denominators (and the unnormalised
+    weighted-V accumulators) are rescaled to the common maximum before adding.
+    Returns ``(O, LSE)`` with ``O = acc / l`` and ``LSE = m + ln l`` (O = 0 and
+    LSE = -inf when no part saw a key).
+    """
+    ms = np.array([p[0] for p in parts], dtype=np.float64)
+    M = ms.max()
+    if not np.isfinite(M):
+        d = np.asarray(parts[0][2]).shape
+        return np.zeros(d), -np.inf
+    L = 0.0
+    acc = 0.0
+    for m, l, a in parts:
+        if np.isfinite(m):
+            w = math.exp(m - M)
+            L = L + l * w
+            acc = acc + np.asarray(a, dtype=np.float64) * w
+    return acc / L, M + math.log(L)
+
+
+def brute_force_attention(q, k, v, causal=False, window_left=-1, scale=None):
+    """Pure-Python loops (no NumPy arithmetic) for tiny shapes.
+
+    Nested lists in, nested lists out: ``O[b][i][h][c]`` and ``LSE[b][h][i]``.
+    Used to check the NumPy oracle on shapes up to about 8 x 8.
+    """
+    B, Nq, Hq, d = len(q), len(q[0]), len(q[0][0]), len(q[0][0][0])
+    Nk, Hkv = len(k[0]), len(k[0][0])
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    group = Hq // Hkv
+    O = [[[[0.0] * d for _ in range(Hq)] for _ in range(Nq)] for _ in range(B)]
+    LSE = [[[-math.inf] * Nq for _ in range(Hq)] for _ in range(B)]
+    for b in range(B):
+        for h in range(Hq):
+            g = h // group
+            for i in range(Nq):
+                qpos = i + Nk - Nq
+                scores = []
+                for j in range(Nk):
+                    ok = True
+                    if causal and j > qpos:
+                        ok = False
+                    if window_left >= 0 and j < qpos - window_left:
+                        ok = False
+                    if ok:
+                        s = 0.0
+                        for c in range(d):
+                            s += float(q[b][i][h][c]) * float(k[b][j][g][c])
+                        scores.append((j, s * scale))
+                if not scores:
+                    continue
+                mx = max(s for _, s in scores)
+                w = [(j, math.exp(s - mx)) for j, s in scores]
+                den = sum(x for _, x in w)
+                for c in range(d):
+                    O[b][i][h][c] = sum(x * float(v[b][j][g][c]) for j, x in w) / den
+                LSE[b][h][i] = mx + math.log(den)
+    return O, LSE
