@@ -1,0 +1,461 @@
+#!/usr/bin/env python
+"""Benchmark of the exact-attention hot path on B200 (one JSON line on rank 0).
+
+A step is one pass of the hot path over one batch of synthetic input:
+  * prefill: one attn_fwd call on the MHA causal prefill workload
+    (B=4, Hq=Hkv=32, N=2048, d=128, bf16 in/out, fp32 LSE) — the headline
+    `value`, in mask-adjusted TFLOP/s;
+  * decode: one attn_decode call (split + combine kernels) on the GQA decode
+    workload (B=64, L=8192, Hq=32, Hkv=8, d=128), reported under "decode" in
+    KV-read GB/s, timed over the same number of steps.
+
+Timing: W untimed warm-up steps, then K steps; each kernel is bracketed by
+CUDA events on the launching stream, preceded by an L2 flush (256 MiB
+memset) and a short device-side sleep so the events measure the kernel
+alone. Barrier + synchronize on both sides; the max over ranks is reported.
+With N > 1 every rank runs its own independent batch (no collective in the
+data path): weak scaling.
+
+`--impl reference` times the fp64 CPU oracle instead (the only other
+implementation of this path), one bounded per-head sample per step.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import attn_inputs as ai  # noqa: E402
+from exact_softmax_attention_03_b200 import metrics  # noqa: E402
+
+METRIC = "attn fwd TFLOP/s (mask-adjusted) & % bf16 peak; decode KV-read GB/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["exact_softmax_attention_03_b200/csrc/" + f for f in
+                  ("attn_api.cu", "sm100_ptx.cuh", "prefill_kernel.cuh", "decode_kernels.cuh")]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["mha2k", "mha8k", "gqa32k"], default="mha2k",
+                    help="prefill workload (default: the MHA causal prefill at N=2048)")
+    ap.add_argument("--decode-splits", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+PREFILL = {"mha2k": ai.MHA_2K, "mha8k": ai.MHA_8K, "gqa32k": ai.GQA_SWA_32K}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS if k in d}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if taken on these sources."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    want = kernel_source_hash()
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 4 and not line.startswith("#") and parts[0] == kernel \
+                    and parts[1] == workload and parts[3] == want:
+                return float(parts[2])
+    return None
+
+
+# ------------------------------------------------------------------ clocks --
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML during a region."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:                         # NVML unavailable: report nothing
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append(mhz)
+                self.reasons |= int(r) & ~0x1
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": [n for b, n in self.REASONS.items() if self.reasons & b],
+                "samples": len(self.samples)}
+
+
+# -------------------------------------------------------------- dist setup --
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ timing --
+
+def timed_kernel_loop(fn, steps, warmup, world, flush=None, sampler=None):
+    """Per-step CUDA-event times (ms) of fn() on the current stream; returns
+    (times, launches of this library inside the timed region)."""
+    import exact_softmax_attention_03_b200 as ea
+    for _ in range(warmup):
+        if flush is not None:
+            flush()
+        fn()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    if sampler is not None:
+        sampler.start()
+    n0 = ea.attn_launch_count()
+    for s, e in ev:
+        if flush is not None:
+            flush()
+        torch.cuda._sleep(100_000)              # hold the stream while the launch is queued
+        s.record()
+        fn()
+        e.record()
+    torch.cuda.synchronize()
+    n1 = ea.attn_launch_count()
+    barrier(world)
+    if sampler is not None:
+        sampler.stop()
+    status = ea.attn_device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status}: {ea.attn_last_error()}")
+    return [s.elapsed_time(e) for s, e in ev], n1 - n0
+
+
+def e2e_loop(step_fn, steps, warmup):
+    """Event-timed region per step including host<->device copies; ms/step."""
+    for _ in range(warmup):
+        step_fn()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(steps):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        step_fn()
+        e.record()
+        e.synchronize()
+        times.append(s.elapsed_time(e))
+    return statistics.mean(times)
+
+
+# ------------------------------------------------------------ cpu baseline --
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_prefill_sample(w, budget_s, q, k, v):
+    """Time the oracle on whole (b, head) problems until ~budget_s of CPU work."""
+    import oracle
+    G = w.Hq // w.Hkv
+    pairs_per_head = metrics.allowed_pairs(w.Nq, w.Nk, w.causal, w.window_left)
+    flops = 0.0
+    heads = 0
+    t0 = time.perf_counter()
+    for b in range(w.B):
+        for hq in range(w.Hq):
+            hk = hq // G
+            oracle.oracle_attention(q[b:b + 1, :, hq:hq + 1], k[b:b + 1, :, hk:hk + 1],
+                                    v[b:b + 1, :, hk:hk + 1], causal=w.causal,
+                                    window_left=w.window_left)
+            flops += 4.0 * w.d * pairs_per_head
+            heads += 1
+            if time.perf_counter() - t0 >= budget_s:
+                break
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return flops / dt / 1e12, heads, dt
+
+
+def cpu_baseline_block(w, q, k, v, budget_s=12.0):
+    tflops, heads, dt = oracle_prefill_sample(w, budget_s, q, k, v)
+    return {"value": tflops, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"fp64 NumPy oracle on {heads} whole (batch, head) problems of "
+                      f"'{w.name}' ({dt:.1f} s), same mask-adjusted FLOP count"}
+
+
+# --------------------------------------------------------------- reference --
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    w = PREFILL[args.workload]
+    q, k, v = ai.make_for(w)
+    import oracle
+    G = w.Hq // w.Hkv
+    flops_head = 4.0 * w.d * metrics.allowed_pairs(w.Nq, w.Nk, w.causal, w.window_left)
+    heads = [(b, h) for b in range(w.B) for h in range(w.Hq)]
+
+    def step(i):
+        b, hq = heads[i % len(heads)]
+        hk = hq // G
+        oracle.oracle_attention(q[b:b + 1, :, hq:hq + 1], k[b:b + 1, :, hk:hk + 1],
+                                v[b:b + 1, :, hk:hk + 1], causal=w.causal, window_left=w.window_left)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(i)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = flops_head / dt / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "seq_len": w.Nq,
+                   "d": w.d, "causal": w.causal, "window_left": w.window_left,
+                   "step": "one whole (batch, head) problem per step"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(),
+                         "kind": "oracle",
+                         "sample": "one (batch, head) problem per step, fp64 NumPy oracle"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# -------------------------------------------------------------------- ours --
+
+def run_ours(args, world, rank, local):
+    import exact_softmax_attention_03_b200 as ea
+    from exact_softmax_attention_03_b200 import build
+    build.build()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    sampler = ClockSampler(torch.cuda.current_device() if world == 1 else local)
+
+    w = PREFILL[args.workload]
+    q_h, k_h, v_h = ai.make_for(w, seed=ai.SEED_Q + 17 * rank)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    o = torch.empty((w.B, w.Nq, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=dev)
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def flush():
+        flush_buf.zero_()
+
+    def fwd():
+        ea.attn_fwd(q, k, v, o=o, lse=lse, causal=w.causal, window_left=w.window_left)
+
+    times, launches = timed_kernel_loop(fwd, args.steps, args.warmup, world, flush, sampler)
+    ms = statistics.mean(times)
+    ms_max = max_over_ranks(ms, world)
+    flops = metrics.attn_flops(w.B, w.Hq, w.Nq, w.Nk, w.d, w.causal, w.window_left)
+    value = world * flops / (ms_max * 1e-3) / 1e12
+    achieved = flops / (ms * 1e-3) / 1e12
+    tiles = metrics.executed_tiles(w.Nq, w.Nk, w.causal, w.window_left) * w.B * w.Hq
+    clocks = sampler.summary()
+
+    # decode leg
+    dw = ai.GQA_DECODE
+    qd_h, kc_h, vc_h = ai.make_decode(dw.B, dw.Hq, dw.Hkv, dw.Nk, dw.d, seed=ai.SEED_Q + 17 * rank)
+    qd, kc, vc = qd_h.to(dev), kc_h.to(dev), vc_h.to(dev)
+    od = torch.empty((dw.B, dw.Hq, dw.d), dtype=torch.bfloat16, device=dev)
+    lsed = torch.empty((dw.B, dw.Hq), dtype=torch.float32, device=dev)
+    ws = torch.empty(ea.attn_decode_workspace_bytes(dw.B, dw.Hq, dw.d, args.decode_splits, dw.Nk),
+                     dtype=torch.uint8, device=dev)
+
+    def dec():
+        ea.attn_decode(qd, kc, vc, o=od, lse=lsed, num_splits=args.decode_splits, workspace=ws)
+
+    # the cache (2.1 GB) is far larger than L2, so no flush between decode steps
+    dtimes, dlaunches = timed_kernel_loop(dec, args.steps, args.warmup, world, None, None)
+    dms = statistics.mean(dtimes)
+    dms_max = max_over_ranks(dms, world)
+    kv_bytes = metrics.decode_kv_bytes([dw.Nk] * dw.B, dw.Hkv, dw.d)
+    d_all = metrics.decode_bytes(dw.B, dw.Hq, dw.Hkv, [dw.Nk] * dw.B, dw.d)
+    d_value = world * kv_bytes / (dms_max * 1e-3) / 1e9
+
+    # end-to-end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        qp, kp, vp = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
+        op = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        lp = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+
+        def e2e_step():
+            q.copy_(qp, non_blocking=True)
+            k.copy_(kp, non_blocking=True)
+            v.copy_(vp, non_blocking=True)
+            ea.attn_fwd(q, k, v, o=o, lse=lse, causal=w.causal, window_left=w.window_left)
+            op.copy_(o, non_blocking=True)
+            lp.copy_(lse, non_blocking=True)
+
+        e_ms = max_over_ranks(e2e_loop(e2e_step, min(args.steps, 30), 2), world)
+        h2d = sum(t.numel() * t.element_size() for t in (qp, kp, vp))
+        d2h = op.numel() * op.element_size() + lp.numel() * lp.element_size()
+        e2e = {"value": world * flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_block(w, q_h, k_h, v_h)
+
+    if rank != 0:
+        return
+    peak_t = peaks["bf16_tflops"]
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_max,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "seq_len": w.Nq,
+                   "d": w.d, "causal": w.causal, "window_left": w.window_left,
+                   "parallelism": f"independent batch per GPU x{world}",
+                   "l2": "256 MiB memset flush before every timed step (outside the events)",
+                   "flop_count": "4*d*allowed (i,j) pairs (mask-adjusted)"},
+        "pct_bf16_peak": 100.0 * achieved / peak_t,
+        "tile_tflops": tiles * 4.0 * 128 * 128 * w.d / (ms * 1e-3) / 1e12,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
+                     "frac": achieved / peak_t, "peak_source": f"{peak_src} bf16_tflops (burst)",
+                     "kernel": "attn_fwd_kernel<128,false>",
+                     "traffic": recorded_traffic("attn_fwd_kernel", args.workload),
+                     "algorithmic_bytes": metrics.attn_fwd_bytes(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d)},
+        "decode": {
+            "workload": dw.name, "value": d_value, "unit": "GB/s", "ms_per_step": dms_max,
+            "roofline": {"bound": "hbm", "achieved": kv_bytes / (dms * 1e-3) / 1e9,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": kv_bytes / (dms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                         "peak_source": f"{peak_src} hbm_gbs",
+                         "kernel": "decode_split_kernel<128,4> + decode_combine_kernel<128>",
+                         "algorithmic_bytes": d_all,
+                         "traffic": recorded_traffic("decode", "decode")},
+            "gpu_launches": dlaunches,
+        },
+        "clocks": clocks,
+        "gpu_launches": launches,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+        "kernel_sources": kernel_source_hash(),
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, world, rank)
+        return
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

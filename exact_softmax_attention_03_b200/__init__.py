@@ -1,0 +1,138 @@
+"""Exact softmax attention for B200 (sm_100a): Python binding of libattn.so.
+
+The functions here carry the C ABI's names (include/attn.h) and only marshal
+torch tensors into pointers, sizes and the current CUDA stream; every step of
+the computation runs in the library's kernels. There is no CPU path: a tensor
+that is not a contiguous CUDA tensor of the right dtype is rejected, and a
+missing library raises.
+
+Layouts: q, o ``[B, Nq, Hq, d]``; k, v ``[B, Nk, Hkv, d]`` (bf16); lse
+``[B, Hq, Nq]`` float32. Decode: q, o ``[B, Hq, d]``; caches
+``[B, Lmax, Hkv, d]``; lse ``[B, Hq]``.
+"""
+
+from __future__ import annotations
+
+import math
+
+import torch
+
+from ._lib import AttnError, check, load  # noqa: F401
+
+__all__ = ["attn_fwd", "attn_fwd_f32o", "attn_decode", "attn_decode_workspace_bytes",
+           "attn_device_status", "attn_last_error", "attn_launch_count", "AttnError"]
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype, ndim: int):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (no CPU path)")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _fwd(q, k, v, o, lse, causal, window_left, scale, stream, f32o):
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k, "k", torch.bfloat16, 4)
+    _need(v, "v", torch.bfloat16, 4)
+    B, Nq, Hq, d = q.shape
+    _, Nk, Hkv, _ = k.shape
+    if k.shape[0] != B or k.shape[3] != d or v.shape != k.shape:
+        raise ValueError("k, v must be [B, Nk, Hkv, d] matching q")
+    out_dtype = torch.float32 if f32o else torch.bfloat16
+    if o is None:
+        o = torch.empty((B, Nq, Hq, d), dtype=out_dtype, device=q.device)
+    _need(o, "o", out_dtype, 4)
+    if tuple(o.shape) != (B, Nq, Hq, d):
+        raise ValueError("o must be [B, Nq, Hq, d]")
+    if lse is not None:
+        _need(lse, "lse", torch.float32, 3)
+        if tuple(lse.shape) != (B, Hq, Nq):
+            raise ValueError("lse must be [B, Hq, Nq]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    fn = load().attn_fwd_f32o if f32o else load().attn_fwd
+    check(fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+             lse.data_ptr() if lse is not None else None,
+             B, Hq, Hkv, Nq, Nk, d, float(scale), int(bool(causal)),
+             int(window_left), _stream_handle(stream)))
+    return o, lse
+
+
+def attn_fwd(q, k, v, o=None, lse=None, causal=False, window_left=-1, scale=None, stream=None):
+    """Forward attention, bf16 output. Returns ``(o, lse)`` (lse as passed, may be None)."""
+    return _fwd(q, k, v, o, lse, causal, window_left, scale, stream, False)
+
+
+def attn_fwd_f32o(q, k, v, o=None, lse=None, causal=False, window_left=-1, scale=None, stream=None):
+    """Forward attention, float32 output. Returns ``(o, lse)``."""
+    return _fwd(q, k, v, o, lse, causal, window_left, scale, stream, True)
+
+
+def attn_decode_workspace_bytes(B: int, Hq: int, d: int, num_splits: int = 0, Lmax: int = 1) -> int:
+    return int(load().attn_decode_workspace_bytes(B, Hq, d, num_splits, Lmax))
+
+
+def attn_decode(q, k_cache, v_cache, o=None, lse=None, seqlens=None, window_left=-1,
+                scale=None, num_splits=0, workspace=None, stream=None):
+    """Single-query decode over a contiguous KV cache. Returns ``(o, lse)``.
+
+    ``workspace`` is a caller-owned CUDA buffer of at least
+    ``attn_decode_workspace_bytes(...)`` bytes; if None, one is allocated here
+    with torch (the library itself never allocates).
+    """
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    _need(v_cache, "v_cache", torch.bfloat16, 4)
+    B, Hq, d = q.shape
+    _, Lmax, Hkv, _ = k_cache.shape
+    if k_cache.shape[0] != B or k_cache.shape[3] != d or v_cache.shape != k_cache.shape:
+        raise ValueError("caches must be [B, Lmax, Hkv, d] matching q")
+    if o is None:
+        o = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q.device)
+    _need(o, "o", torch.bfloat16, 3)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, 2)
+    if seqlens is not None:
+        _need(seqlens, "seqlens", torch.int32, 1)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    need = attn_decode_workspace_bytes(B, Hq, d, num_splits, Lmax)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if not workspace.is_cuda:
+        raise ValueError("workspace must be a CUDA tensor")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    check(load().attn_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), o.data_ptr(),
+                             lse.data_ptr() if lse is not None else None,
+                             seqlens.data_ptr() if seqlens is not None else None,
+                             B, Hq, Hkv, Lmax, d, float(scale), int(window_left), int(num_splits),
+                             workspace.data_ptr(), ws_bytes, _stream_handle(stream)))
+    return o, lse
+
+
+def attn_device_status(stream=None) -> int:
+    """Synchronise the stream, read and clear the device timeout word (0 = ok)."""
+    return int(load().attn_device_status(_stream_handle(stream)))
+
+
+def attn_last_error() -> str:
+    msg = load().attn_last_error()
+    return msg.decode() if msg else ""
+
+
+def attn_launch_count() -> int:
+    return int(load().attn_launch_count())

@@ -1,0 +1,322 @@
+// attn_api.cu — the C ABI declared in include/attn.h: host-side argument
+// validation, TMA descriptor encoding, launch configuration and error codes.
+// Compiled as a single translation unit with the kernels it launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/attn.h"
+#include "decode_kernels.cuh"
+#include "prefill_kernel.cuh"
+
+namespace {
+
+thread_local char g_err[512] = "";
+std::atomic<unsigned long long> g_launches{0};
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int ok() {
+  g_err[0] = '\0';
+  return ATTN_OK;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// The device current on this thread must be a compute-capability 10.0 part
+// (sm_100a code only). Result cached per device ordinal.
+int check_device(int* dev_out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  static std::atomic<int> cache[64];   // 0 unknown, 1 ok, 2 unsupported
+  if (dev >= 0 && dev < 64) {
+    const int c = cache[dev].load();
+    if (c == 1) { *dev_out = dev; return ATTN_OK; }
+    if (c == 2) return fail(ATTN_ERR_UNSUPPORTED, "device %d is not sm_100", dev);
+  }
+  int major = 0, minor = 0;
+  if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
+    return fail(ATTN_ERR_CUDA, "cudaDeviceGetAttribute: %s", cudaGetErrorString(e));
+  const bool good = (major == 10 && minor == 0);
+  if (dev >= 0 && dev < 64) cache[dev].store(good ? 1 : 2);
+  if (!good) return fail(ATTN_ERR_UNSUPPORTED, "device %d is sm_%d%d, need sm_100", dev, major, minor);
+  *dev_out = dev;
+  return ATTN_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// 4-D view {d, H, N, B} of a contiguous bf16 [B, N, H, d] tensor; box
+// {64, 1, 128, 1} with 128-byte swizzle (one 128-row x 128-byte block).
+int make_map(CUtensorMap* map, const void* base, int d, int H, int N, int B) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[4] = {cuuint64_t(d), cuuint64_t(H), cuuint64_t(N), cuuint64_t(B)};
+  cuuint64_t strides[3] = {cuuint64_t(d) * 2, cuuint64_t(H) * d * 2, cuuint64_t(N) * H * d * 2};
+  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return ATTN_OK;
+}
+
+bool finite_pos(float x) { return std::isfinite(x) && x > 0.f; }
+
+constexpr long long kMaxIndex = (1ll << 31) - 1;
+
+int validate_fwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                 int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal) {
+  if (!q || !k || !v || !o) return fail(ATTN_ERR_INVALID_ARG, "q, k, v and o must be non-null");
+  if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1)
+    return fail(ATTN_ERR_INVALID_ARG, "B, Hq, Hkv, Nq, Nk must be >= 1");
+  if (Hq % Hkv != 0) return fail(ATTN_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
+  if (d != 64 && d != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim %d not in {64, 128}", d);
+  if (!finite_pos(scale)) return fail(ATTN_ERR_INVALID_ARG, "scale must be finite and > 0");
+  if (causal != 0 && causal != 1) return fail(ATTN_ERR_INVALID_ARG, "causal must be 0 or 1");
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16))
+    return fail(ATTN_ERR_INVALID_ARG, "q, k, v, o must be 16-byte aligned");
+  if (lse && !aligned(lse, 4)) return fail(ATTN_ERR_INVALID_ARG, "lse must be 4-byte aligned");
+  // index arithmetic in the kernels uses 32-bit rows and positions
+  if (static_cast<long long>(B) * Nq > kMaxIndex || static_cast<long long>(B) * Nk > kMaxIndex ||
+      static_cast<long long>(B) * Hq > kMaxIndex)
+    return fail(ATTN_ERR_INVALID_ARG, "sizes too large");
+  return ATTN_OK;
+}
+
+template <int D, bool F32OUT>
+int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+               int Hkv, int Nq, int Nk, float scale, int causal, int window_left,
+               cudaStream_t stream, int dev) {
+  using L = attn::FwdLayout<D>;
+  CUtensorMap mq, mk, mv;
+  int rc;
+  if ((rc = make_map(&mq, q, D, Hq, Nq, B)) != ATTN_OK) return rc;
+  if ((rc = make_map(&mk, k, D, Hkv, Nk, B)) != ATTN_OK) return rc;
+  if ((rc = make_map(&mv, v, D, Hkv, Nk, B)) != ATTN_OK) return rc;
+
+  attn::FwdParams p{};
+  p.o = o;
+  p.lse = lse;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Nq = Nq; p.Nk = Nk;
+  p.causal = causal;
+  p.window_left = window_left < 0 ? -1 : window_left;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const int G = Hq / Hkv;
+  p.pair_heads = (G % 2 == 0) ? 1 : 0;
+  p.n_qblk = (Nq + 127) / 128;
+  if (p.pair_heads) {
+    p.n_units = p.n_qblk;
+    p.n_bh = B * Hkv * (G / 2);
+  } else {
+    p.n_units = (p.n_qblk + 1) / 2;
+    p.n_bh = B * Hq;
+  }
+  const long long grid = static_cast<long long>(p.n_units) * p.n_bh;
+  if (grid > kMaxIndex) return fail(ATTN_ERR_INVALID_ARG, "problem too large for one launch");
+
+  static std::atomic<unsigned long long> attr_set{0};   // per-device bit
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(attr_set.load() & bit)) {
+    cudaError_t e = cudaFuncSetAttribute(attn::attn_fwd_kernel<D, F32OUT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_ALLOC);
+    if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    attr_set.fetch_or(bit);
+  }
+  attn::attn_fwd_kernel<D, F32OUT><<<unsigned(grid), attn::kFwdThreads, L::SMEM_ALLOC, stream>>>(mq, mk, mv, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "attn_fwd launch: %s", cudaGetErrorString(e));
+  g_launches.fetch_add(1);
+  return ok();
+}
+
+int fwd_entry(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+              int Hkv, int Nq, int Nk, int d, float scale, int causal, int window_left,
+              cudaStream_t stream, bool f32out) {
+  int rc = validate_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal);
+  if (rc != ATTN_OK) return rc;
+  int dev = 0;
+  if ((rc = check_device(&dev)) != ATTN_OK) return rc;
+  if (d == 128) {
+    return f32out ? launch_fwd<128, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, window_left, stream, dev)
+                  : launch_fwd<128, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, window_left, stream, dev);
+  }
+  return f32out ? launch_fwd<64, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, window_left, stream, dev)
+                : launch_fwd<64, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, window_left, stream, dev);
+}
+
+// ------------------------------------------------------------------ decode --
+
+constexpr int kNumSMs = 148;
+
+int decode_group_tile(int G) {
+  if (G % 4 == 0) return 4;
+  if (G % 2 == 0) return 2;
+  return 1;
+}
+
+// Split count chosen from sizes alone (so the workspace size needs no Hkv):
+// enough CTAs for several waves over the SMs, each streaming >= 256 keys.
+int auto_splits(int B, int Hq, int Lmax) {
+  const long long items = std::max(1ll, (static_cast<long long>(B) * Hq + 3) / 4);
+  long long s = (static_cast<long long>(kNumSMs) * 8 + items - 1) / items;
+  const long long cap = std::max(1, (Lmax + 255) / 256);
+  s = std::min(std::max(s, 1ll), cap);
+  return static_cast<int>(std::min(s, 256ll));
+}
+
+struct DecodeShape {
+  int S;
+  int chunk;
+  size_t acc_bytes, ml_bytes, total;
+};
+
+DecodeShape decode_shape(int B, int Hq, int d, int num_splits, int Lmax) {
+  DecodeShape s{};
+  int S = num_splits > 0 ? num_splits : auto_splits(B, Hq, Lmax);
+  if (S > Lmax) S = Lmax;
+  const int quantum = (d == 128) ? 32 : 64;         // keys per CTA block of passes
+  int chunk = (Lmax + S - 1) / S;
+  chunk = (chunk + quantum - 1) / quantum * quantum;
+  S = (Lmax + chunk - 1) / chunk;
+  s.S = S;
+  s.chunk = chunk;
+  auto round256 = [](size_t x) { return (x + 255) / 256 * 256; };
+  s.acc_bytes = round256(static_cast<size_t>(B) * Hq * S * d * sizeof(float));
+  s.ml_bytes = round256(static_cast<size_t>(B) * Hq * S * 2 * sizeof(float));
+  s.total = s.acc_bytes + s.ml_bytes;
+  return s;
+}
+
+template <int D, int GT>
+void launch_decode_kernels(const attn::DecodeParams& p, cudaStream_t stream) {
+  const int G = p.Hq / p.Hkv;
+  dim3 grid_split(p.S, p.Hkv * (G / GT), p.B);
+  attn::decode_split_kernel<D, GT><<<grid_split, attn::kDecodeThreads, 0, stream>>>(p);
+  const int n = p.B * p.Hq;
+  attn::decode_combine_kernel<D><<<(n + 3) / 4, 128, 0, stream>>>(p);
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+             int Hkv, int Nq, int Nk, int d, float scale, int causal, int window_left,
+             cudaStream_t stream) {
+  return fwd_entry(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, window_left, stream, false);
+}
+
+int attn_fwd_f32o(const void* q, const void* k, const void* v, float* o, float* lse, int B, int Hq,
+                  int Hkv, int Nq, int Nk, int d, float scale, int causal, int window_left,
+                  cudaStream_t stream) {
+  return fwd_entry(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, window_left, stream, true);
+}
+
+size_t attn_decode_workspace_bytes(int B, int Hq, int d, int num_splits, int Lmax) {
+  if (B < 1 || Hq < 1 || Lmax < 1 || (d != 64 && d != 128) || num_splits < 0) return 0;
+  return decode_shape(B, Hq, d, num_splits, Lmax).total;
+}
+
+int attn_decode(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
+                const int* seqlens, int B, int Hq, int Hkv, int Lmax, int d, float scale,
+                int window_left, int num_splits, void* workspace, size_t workspace_bytes,
+                cudaStream_t stream) {
+  if (!q || !k_cache || !v_cache || !o)
+    return fail(ATTN_ERR_INVALID_ARG, "q, k_cache, v_cache and o must be non-null");
+  if (B < 1 || Hq < 1 || Hkv < 1 || Lmax < 1)
+    return fail(ATTN_ERR_INVALID_ARG, "B, Hq, Hkv, Lmax must be >= 1");
+  if (Hq % Hkv != 0) return fail(ATTN_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
+  if (d != 64 && d != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim %d not in {64, 128}", d);
+  if (!finite_pos(scale)) return fail(ATTN_ERR_INVALID_ARG, "scale must be finite and > 0");
+  if (num_splits < 0) return fail(ATTN_ERR_INVALID_ARG, "num_splits must be >= 0");
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(o, 16))
+    return fail(ATTN_ERR_INVALID_ARG, "q, k_cache, v_cache, o must be 16-byte aligned");
+  if (lse && !aligned(lse, 4)) return fail(ATTN_ERR_INVALID_ARG, "lse must be 4-byte aligned");
+  if (seqlens && !aligned(seqlens, 4)) return fail(ATTN_ERR_INVALID_ARG, "seqlens must be 4-byte aligned");
+  if (static_cast<long long>(B) * Lmax > kMaxIndex || static_cast<long long>(B) * Hq > kMaxIndex)
+    return fail(ATTN_ERR_INVALID_ARG, "sizes too large");
+  const DecodeShape sh = decode_shape(B, Hq, d, num_splits, Lmax);
+  if (workspace == nullptr || workspace_bytes < sh.total)
+    return fail(ATTN_ERR_WORKSPACE, "workspace of %zu bytes needed, got %zu", sh.total,
+                workspace == nullptr ? size_t(0) : workspace_bytes);
+  if (!aligned(workspace, 256)) return fail(ATTN_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  int dev = 0;
+  int rc = check_device(&dev);
+  if (rc != ATTN_OK) return rc;
+
+  attn::DecodeParams p{};
+  p.q = static_cast<const uint16_t*>(q);
+  p.k = static_cast<const uint16_t*>(k_cache);
+  p.v = static_cast<const uint16_t*>(v_cache);
+  p.o = static_cast<uint16_t*>(o);
+  p.lse = lse;
+  p.seqlens = seqlens;
+  p.ws_acc = static_cast<float*>(workspace);
+  p.ws_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) + sh.acc_bytes);
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Lmax = Lmax;
+  p.S = sh.S;
+  p.chunk = sh.chunk;
+  p.window_left = window_left < 0 ? -1 : window_left;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const int GT = decode_group_tile(Hq / Hkv);
+  if (d == 128) {
+    if (GT == 4) launch_decode_kernels<128, 4>(p, stream);
+    else if (GT == 2) launch_decode_kernels<128, 2>(p, stream);
+    else launch_decode_kernels<128, 1>(p, stream);
+  } else {
+    if (GT == 4) launch_decode_kernels<64, 4>(p, stream);
+    else if (GT == 2) launch_decode_kernels<64, 2>(p, stream);
+    else launch_decode_kernels<64, 1>(p, stream);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "attn_decode launch: %s", cudaGetErrorString(e));
+  g_launches.fetch_add(2);
+  return ok();
+}
+
+const char* attn_last_error(void) { return g_err; }
+
+int attn_device_status(cudaStream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "stream: %s", cudaGetErrorString(e));
+  int val = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&val, attn::g_attn_status, sizeof(int));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(attn::g_attn_status, &zero, sizeof(int));
+  if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "status word: %s", cudaGetErrorString(e));
+  if (val != 0) return fail(ATTN_ERR_TIMEOUT, "a device-side wait timed out");
+  return ok();
+}
+
+unsigned long long attn_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"

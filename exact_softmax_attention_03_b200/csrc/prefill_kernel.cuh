@@ -1,0 +1,465 @@
+// prefill_kernel.cuh — exact attention forward pass on sm_100a tensor cores.
+//
+// The tiled loop of "Attention Is O(n²): FlashAttention vs Linear Attention",
+// section "FlashAttention — Same FLOPs, Linear Memory": for each query block,
+// walk the key/value blocks, keep a running row maximum and running sum, rescale
+// the accumulator when the maximum moves, divide by the sum at the end. The
+// score tile never leaves the SM: it lives in tensor memory (TMEM).
+//
+// One CTA (384 threads) owns two 128-row query tiles that share every K/V tile:
+//   * two heads of one K/V group at the same rows when Hq / Hkv is even
+//     (the grouped-query map of "Chapter 3: MHA Limitations, MQA, GQA, and
+//     FlashAttention", section 3.3, so each K/V tile is loaded once for both),
+//   * otherwise two consecutive row blocks of one head.
+// Warp roles:
+//   warps 0-3  softmax for tile 0 (thread = query row = TMEM lane)
+//   warps 4-7  softmax for tile 1
+//   warp 8     tensor-core issuer (one lane): S_t = Q_t K_jᵀ and O_t += P_t V_j
+//   warp 9     TMA producer (one lane): Q once, then K_j / V_j through a ring
+//   warps 10-11 idle (register budget only)
+// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D), O1 after it.
+// P_t is written as bf16 pairs over the first 64 columns of S_t and read by
+// the P·V product straight from TMEM.
+//
+// Masks ("Modern Attention ...", section 4 for the window; bottom-right causal
+// alignment): key blocks wholly outside a tile's allowed range are skipped;
+// boundary blocks are masked element by element in the softmax warps.
+// Every mbarrier wait is bounded (sm100_ptx.cuh); on a timeout the CTA stops
+// issuing work, drains what it issued, frees TMEM and exits.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include "sm100_ptx.cuh"
+
+namespace attn {
+
+template <int D>
+struct FwdLayout {
+  static constexpr int BM = 128;                       // query rows per tile
+  static constexpr int BN = 128;                       // keys per K/V tile
+  static constexpr int TILE = BM * D * 2;              // bytes of a 128 x D bf16 tile
+  static constexpr int HALF = 128 * 128;               // one 128-row x 64-col swizzle block
+  static constexpr int STAGES = (D == 128) ? 2 : 4;    // K/V ring depth
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + 2 * TILE;
+  static constexpr int OFF_V = OFF_K + STAGES * TILE;
+  static constexpr int OFF_BAR = OFF_V + STAGES * TILE;
+  // barrier indices
+  static constexpr int B_Q = 0;
+  static constexpr int B_KF = 1;                        // + stage
+  static constexpr int B_KE = B_KF + STAGES;
+  static constexpr int B_VF = B_KE + STAGES;
+  static constexpr int B_VE = B_VF + STAGES;
+  static constexpr int B_SF = B_VE + STAGES;            // + tile
+  static constexpr int B_PF = B_SF + 2;
+  static constexpr int B_OD = B_PF + 2;
+  static constexpr int B_DRAIN = B_OD + 2;
+  static constexpr int NBAR = B_DRAIN + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // [0] TMEM base, [1] abort flag
+  static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int SMEM_ALLOC = BYTES + 1024;       // slack for 1024-byte alignment
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
+  static constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, 0);
+  static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, 1);
+};
+
+struct FwdParams {
+  void* o;                 // [B, Nq, Hq, D] bf16 or f32
+  float* lse;              // [B, Hq, Nq] or null
+  int B, Hq, Hkv, Nq, Nk;
+  int causal, window_left;
+  float scale;             // softmax scale
+  float scale_log2;        // scale * log2(e)
+  int pair_heads;          // 1: tiles = two heads of a group at the same rows
+  int n_qblk;              // ceil(Nq / 128)
+  int n_units;             // row units per (b, head-or-pair)
+  int n_bh;                // number of (b, head-or-pair) combinations
+};
+
+constexpr int kFwdThreads = 384;
+
+struct TileInfo {
+  int hq, row0, active;    // query head, first row, any row < Nq
+  int blo, bhi;            // key blocks [blo, bhi); empty if bhi <= blo
+};
+
+__device__ __forceinline__ void tile_range(const FwdParams& p, TileInfo& t) {
+  t.blo = 0;
+  t.bhi = 0;
+  if (!t.active) return;
+  const int r_last = min(t.row0 + 127, p.Nq - 1);
+  const int qf = t.row0 + p.Nk - p.Nq;
+  const int ql = r_last + p.Nk - p.Nq;
+  const int hi = p.causal ? min(p.Nk, ql + 1) : p.Nk;
+  const int lo = p.window_left >= 0 ? max(0, qf - p.window_left) : 0;
+  if (hi <= lo) return;
+  t.blo = lo / 128;
+  t.bhi = (hi - 1) / 128 + 1;
+}
+
+__device__ __forceinline__ bool tile_has(const TileInfo& t, int j) {
+  return j >= t.blo && j < t.bhi;
+}
+
+// Whether key block j needs element-wise masking for this tile's rows.
+__device__ __forceinline__ bool block_needs_mask(const FwdParams& p, const TileInfo& t, int j) {
+  const int kb0 = j * 128, kb1 = kb0 + 127;
+  const int r_last = min(t.row0 + 127, p.Nq - 1);
+  const int qf = t.row0 + p.Nk - p.Nq;
+  const int ql = r_last + p.Nk - p.Nq;
+  return kb1 >= p.Nk || (p.causal && kb1 > qf) || (p.window_left >= 0 && kb0 < ql - p.window_left);
+}
+
+template <int D>
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem) {
+  using L = FwdLayout<D>;
+#pragma unroll
+  for (int k = 0; k < D / 16; ++k) {
+    const uint32_t off = (k / 4) * L::HALF + (k % 4) * 32;
+    const uint64_t a = smem_desc_sw128(q_smem + off, 16, 1024);
+    const uint64_t b = smem_desc_sw128(k_smem + off, 16, 1024);
+    mma_ss(d_tmem, a, b, L::IDESC_QK, k > 0 ? 1u : 0u);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_smem,
+                                         bool accumulate) {
+  using L = FwdLayout<D>;
+#pragma unroll
+  for (int k = 0; k < 128 / 16; ++k) {
+    const uint64_t b = smem_desc_sw128(v_smem + k * 16 * 128, L::HALF, 1024);
+    mma_ts(d_tmem, p_tmem + 8 * k, b, L::IDESC_PV, (accumulate || k > 0) ? 1u : 0u);
+  }
+}
+
+template <int D, bool F32OUT>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  using L = FwdLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  auto bar = [&](int i) -> uint32_t { return sb + L::OFF_BAR + 8u * uint32_t(i); };
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work item -----------------------------------------------------------
+  const int unit = p.n_units - 1 - int(blockIdx.x) / p.n_bh;   // longest rows first
+  const int bh = int(blockIdx.x) % p.n_bh;
+  int b, hkv;
+  TileInfo tile[2];
+  if (p.pair_heads) {
+    const int G = p.Hq / p.Hkv;
+    const int pairs = G / 2;
+    b = bh / (p.Hkv * pairs);
+    const int rem = bh % (p.Hkv * pairs);
+    hkv = rem / pairs;
+    const int pr = rem % pairs;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      tile[t].hq = hkv * G + 2 * pr + t;
+      tile[t].row0 = unit * 128;
+    }
+  } else {
+    b = bh / p.Hq;
+    const int hq = bh % p.Hq;
+    hkv = hq / (p.Hq / p.Hkv);
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      tile[t].hq = hq;
+      tile[t].row0 = (2 * unit + t) * 128;
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    tile[t].active = tile[t].row0 < p.Nq;
+    tile_range(p, tile[t]);
+  }
+  const bool ne0 = tile[0].bhi > tile[0].blo, ne1 = tile[1].bhi > tile[1].blo;
+  int ublo = 0, ubhi = 0;
+  if (ne0 || ne1) {
+    ublo = ne0 ? (ne1 ? min(tile[0].blo, tile[1].blo) : tile[0].blo) : tile[1].blo;
+    ubhi = ne0 ? (ne1 ? max(tile[0].bhi, tile[1].bhi) : tile[0].bhi) : tile[1].bhi;
+  }
+  const int U = ubhi - ublo;              // key blocks visited, in descending order
+
+  // ---- setup ---------------------------------------------------------------
+  if (threadIdx.x == 0) {
+    mbar_init(bar(L::B_Q), 1);
+    for (int s = 0; s < L::STAGES; ++s) {
+      mbar_init(bar(L::B_KF + s), 1);
+      mbar_init(bar(L::B_KE + s), 1);
+      mbar_init(bar(L::B_VF + s), 1);
+      mbar_init(bar(L::B_VE + s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(L::B_SF + t), 1);
+      mbar_init(bar(L::B_PF + t), 128);
+      mbar_init(bar(L::B_OD + t), 1);
+    }
+    mbar_init(bar(L::B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(smem_u32(tmem_holder), L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp < 8) {
+    // ======================= softmax warpgroups ==============================
+    const int t = warp >> 2;
+    const TileInfo& T = tile[t];
+    const int row = int(threadIdx.x) - 128 * t;
+    const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_off + (t ? L::COL_S1 : L::COL_S0);
+    const uint32_t tO = tmem + lane_off + (t ? L::COL_O1 : L::COL_O0);
+    const int r = T.row0 + row;
+    const int qpos = r + p.Nk - p.Nq;
+    const float c2 = p.scale_log2;
+    float m = -CUDART_INF_F;                // running max (raw score units)
+    float l = 0.f;                          // running sum of exp2((s - m) * c2)
+    int count = 0;
+    bool ok = true;
+    for (int j = T.bhi - 1; j >= T.blo; --j) {
+      bool w = mbar_wait(bar(L::B_SF + t), uint32_t(count & 1), abort_flag);
+      if (w && count > 0) w = mbar_wait(bar(L::B_OD + t), uint32_t((count - 1) & 1), abort_flag);
+      if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+      tc_fence_after();
+
+      uint32_t sr[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, sr + 32 * c);
+      tmem_wait_ld();
+      float s[128];
+#pragma unroll
+      for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
+
+      if (block_needs_mask(p, T, j)) {
+        const int kb0 = j * 128;
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          const int key = kb0 + c;
+          const bool allowed = key < p.Nk && (!p.causal || key <= qpos) &&
+                               (p.window_left < 0 || key >= qpos - p.window_left);
+          if (!allowed) s[c] = -CUDART_INF_F;
+        }
+      }
+      float mb = s[0];
+#pragma unroll
+      for (int c = 1; c < 128; ++c) mb = fmaxf(mb, s[c]);
+      // Lazy rescale: keep the old maximum while the new one exceeds it by at
+      // most 8 in log2 units (P values stay <= 256); the final O / l is exact
+      // whichever maximum was used.
+      const float m_new = fmaxf(m, mb);
+      const bool rescale = (m_new - m) * c2 > 8.0f;       // false when both are -inf
+      float alpha = 1.f;
+      if (rescale) {
+        alpha = ex2_approx((m - m_new) * c2);              // 0 when m was -inf
+        m = m_new;
+      }
+      const float mo = (m == -CUDART_INF_F) ? 0.f : m * c2;
+      float ls = 0.f;
+      uint32_t pk[64];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const float p0 = ex2_approx(fmaf(s[2 * c], c2, -mo));
+        const float p1 = ex2_approx(fmaf(s[2 * c + 1], c2, -mo));
+        ls += p0 + p1;
+        pk[c] = pack_bf16x2(p0, p1);
+      }
+      l = fmaf(l, alpha, ls);
+      tmem_st32(tS, pk);
+      tmem_st32(tS + 32, pk + 32);
+
+      if (count > 0 && __any_sync(0xffffffffu, rescale)) {
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * c, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(tO + 32 * c, o);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(L::B_PF + t));
+      ++count;
+    }
+
+    // ---- epilogue: O / l and LSE -------------------------------------------
+    if (T.active) {
+      bool have = ok && count > 0;
+      if (have) have = mbar_wait(bar(L::B_OD + t), uint32_t((count - 1) & 1), abort_flag);
+      have = __all_sync(0xffffffffu, have);
+      if (have) tc_fence_after();
+      const bool store = r < p.Nq;
+      const float inv = (l > 0.f) ? 1.f / l : 0.f;
+      const size_t obase = ((size_t(b) * p.Nq + r) * p.Hq + T.hq) * D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        if (have) {
+          tmem_ld32(tO + 32 * c, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = 0u;
+        }
+        if (store) {
+          if constexpr (F32OUT) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + obase + 32 * c);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              dst[e] = make_float4(__uint_as_float(o[4 * e]) * inv, __uint_as_float(o[4 * e + 1]) * inv,
+                                   __uint_as_float(o[4 * e + 2]) * inv, __uint_as_float(o[4 * e + 3]) * inv);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) + obase + 32 * c);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(o[8 * e + 0]) * inv, __uint_as_float(o[8 * e + 1]) * inv);
+              w.y = pack_bf16x2(__uint_as_float(o[8 * e + 2]) * inv, __uint_as_float(o[8 * e + 3]) * inv);
+              w.z = pack_bf16x2(__uint_as_float(o[8 * e + 4]) * inv, __uint_as_float(o[8 * e + 5]) * inv);
+              w.w = pack_bf16x2(__uint_as_float(o[8 * e + 6]) * inv, __uint_as_float(o[8 * e + 7]) * inv);
+              dst[e] = w;
+            }
+          }
+        }
+      }
+      if (store && p.lse != nullptr) {
+        p.lse[(size_t(b) * p.Hq + T.hq) * p.Nq + r] =
+            (l > 0.f) ? fmaf(m, p.scale, __log2f(l) * 0.6931471805599453f) : -CUDART_INF_F;
+      }
+    }
+  } else if (warp == 8) {
+    // ======================= tensor-core issuer ==============================
+    if (lane == 0 && U > 0) {
+      const uint32_t q0 = sb + L::OFF_Q, q1 = sb + L::OFF_Q + L::TILE;
+      const uint32_t dS0 = tmem + L::COL_S0, dS1 = tmem + L::COL_S1;
+      const uint32_t dO0 = tmem + L::COL_O0, dO1 = tmem + L::COL_O1;
+      int pv0 = 0, pv1 = 0;                 // P·V products issued per tile
+      int prev_j = -1, prev_slot = 0;
+      bool alive = mbar_wait(bar(L::B_Q), 0, abort_flag);
+      if (alive) tc_fence_after();
+      for (int it = 0; alive && it < U; ++it) {
+        const int j = ubhi - 1 - it;
+        const int slot = it % L::STAGES;
+        const uint32_t ph = uint32_t(it / L::STAGES) & 1u;
+        if (!(alive = mbar_wait(bar(L::B_KF + slot), ph, abort_flag))) break;
+        tc_fence_after();
+        const uint32_t ks = sb + L::OFF_K + slot * L::TILE;
+        if (tile_has(tile[0], j)) {
+          issue_qk<D>(dS0, q0, ks);
+          tc_commit(bar(L::B_SF + 0));
+        }
+        if (it > 0) {
+          if (tile_has(tile[1], prev_j)) {
+            if (!(alive = mbar_wait(bar(L::B_PF + 1), uint32_t(pv1 & 1), abort_flag))) break;
+            tc_fence_after();
+            issue_pv<D>(dO1, dS1, sb + L::OFF_V + prev_slot * L::TILE, pv1 > 0);
+            tc_commit(bar(L::B_OD + 1));
+            ++pv1;
+          }
+          tc_commit(bar(L::B_VE + prev_slot));
+        }
+        if (tile_has(tile[1], j)) {
+          issue_qk<D>(dS1, q1, ks);
+          tc_commit(bar(L::B_SF + 1));
+        }
+        tc_commit(bar(L::B_KE + slot));
+        if (!(alive = mbar_wait(bar(L::B_VF + slot), ph, abort_flag))) break;
+        tc_fence_after();
+        if (tile_has(tile[0], j)) {
+          if (!(alive = mbar_wait(bar(L::B_PF + 0), uint32_t(pv0 & 1), abort_flag))) break;
+          tc_fence_after();
+          issue_pv<D>(dO0, dS0, sb + L::OFF_V + slot * L::TILE, pv0 > 0);
+          tc_commit(bar(L::B_OD + 0));
+          ++pv0;
+        }
+        prev_j = j;
+        prev_slot = slot;
+      }
+      if (alive && prev_j >= 0) {
+        if (tile_has(tile[1], prev_j)) {
+          alive = mbar_wait(bar(L::B_PF + 1), uint32_t(pv1 & 1), abort_flag);
+          if (alive) {
+            tc_fence_after();
+            issue_pv<D>(dO1, dS1, sb + L::OFF_V + prev_slot * L::TILE, pv1 > 0);
+            tc_commit(bar(L::B_OD + 1));
+            ++pv1;
+          }
+        }
+        tc_commit(bar(L::B_VE + prev_slot));
+      }
+      // drain: every issued tensor-core operation completes before teardown
+      tc_commit(bar(L::B_DRAIN));
+      mbar_wait(bar(L::B_DRAIN), 0, nullptr);
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ======================= TMA producer ====================================
+    if (lane == 0 && U > 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      mbar_arrive_expect_tx(bar(L::B_Q), 2 * L::TILE);
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_4d(sb + L::OFF_Q + t * L::TILE + c * L::HALF, &tmQ, bar(L::B_Q), c * 64,
+                      tile[t].hq, tile[t].row0, b);
+      int issued_k = 0, issued_v = 0;
+      for (int it = 0; it < U; ++it) {
+        const int j = ubhi - 1 - it;
+        const int slot = it % L::STAGES;
+        const uint32_t ph = uint32_t(it / L::STAGES) & 1u;
+        if (!mbar_wait(bar(L::B_KE + slot), ph ^ 1u, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(L::B_KF + slot), L::TILE);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_4d(sb + L::OFF_K + slot * L::TILE + c * L::HALF, &tmK, bar(L::B_KF + slot),
+                      c * 64, hkv, j * 128, b);
+        issued_k = it + 1;
+        if (!mbar_wait(bar(L::B_VE + slot), ph ^ 1u, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(L::B_VF + slot), L::TILE);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_4d(sb + L::OFF_V + slot * L::TILE + c * L::HALF, &tmV, bar(L::B_VF + slot),
+                      c * 64, hkv, j * 128, b);
+        issued_v = it + 1;
+      }
+      // Make sure no copy is still landing in shared memory at exit: wait for
+      // the most recent phase of every stage (already complete normally).
+      mbar_wait(bar(L::B_Q), 0, nullptr);
+      for (int it = max(0, issued_k - L::STAGES); it < issued_k; ++it)
+        mbar_wait(bar(L::B_KF + it % L::STAGES), uint32_t(it / L::STAGES) & 1u, nullptr);
+      for (int it = max(0, issued_v - L::STAGES); it < issued_v; ++it)
+        mbar_wait(bar(L::B_VF + it % L::STAGES), uint32_t(it / L::STAGES) & 1u, nullptr);
+    }
+    __syncwarp();
+  }
+
+  // ---- teardown --------------------------------------------------------------
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::TMEM_COLS);
+  }
+}
+
+}  // namespace attn

@@ -1,0 +1,128 @@
+/*
+ * attn.h — C ABI of the exact softmax attention library (libattn.so), sm_100a.
+ *
+ * Operation (all entry points):  O = softmax(scale * Q Kᵀ + mask) V, computed
+ * tile by tile with an online softmax so the score matrix never reaches device
+ * memory, plus the per-row natural log-sum-exp of the scaled, masked scores.
+ *   - Plain definition: "Attention Is O(n²): FlashAttention vs Linear
+ *     Attention", section "Why Attention Is O(n²)".
+ *   - Tiled loop with running max / running sum / rescaled accumulator: same
+ *     page, section "FlashAttention — Same FLOPs, Linear Memory"; the online
+ *     softmax of "Modern Attention: MQA, GQA, FlashAttention, Sliding Window
+ *     and RoPE", section 3.
+ *   - Grouped-query heads: query head h reads K/V head h / (Hq / Hkv)
+ *     ("Chapter 3: MHA Limitations, MQA, GQA, and FlashAttention", section 3.3).
+ *   - Sliding window: "Modern Attention ...", section 4.
+ *   - Decode over a KV cache, combined from key-split partial states by the
+ *     merge rule of "Chapter 3 ...", section 3.5.
+ *
+ * Mask convention. Query row i sits at key position qpos(i) = i + Nk - Nq
+ * (bottom-right alignment). Key j is allowed iff 0 <= j < Nk and
+ *   j <= qpos(i)                  when causal != 0, and
+ *   j >= qpos(i) - window_left    when window_left >= 0.
+ * window_left counts keys strictly before the query's own position, so a
+ * window of the "last W tokens" is window_left = W - 1. A negative
+ * window_left means no window; a window without causal limits the left side
+ * only. A row with no allowed key gets O = 0 and LSE = -inf.
+ *
+ * Layouts (row-major, contiguous, element strides implied by the shapes):
+ *   Q, O : [B, Nq, Hq, d]      K, V : [B, Nk, Hkv, d]      LSE : [B, Hq, Nq]
+ * Q/K/V are bfloat16; O is bfloat16 (attn_fwd) or float32 (attn_fwd_f32o);
+ * LSE is float32 in natural-log units of the scaled scores.
+ *
+ * Ownership. The caller allocates and owns every buffer (device memory),
+ * including the decode workspace; the library never allocates or frees device
+ * memory. All calls are asynchronous on `stream` (may be NULL = legacy default
+ * stream) and never synchronise, except attn_device_status.
+ *
+ * Errors. Every entry point validates its arguments on the host first; on any
+ * error it returns a non-zero attn_status, launches nothing, and records a
+ * message readable with attn_last_error() (thread-local).
+ */
+#ifndef ATTN_H_
+#define ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misalignment, Hq % Hkv != 0, ... */
+  ATTN_ERR_UNSUPPORTED = 2,   /* device is not sm_100, or head dim not in {64, 128} */
+  ATTN_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed (message has the code) */
+  ATTN_ERR_TIMEOUT = 4,       /* a bounded device-side wait gave up (see attn_device_status) */
+  ATTN_ERR_WORKSPACE = 5      /* decode workspace missing or smaller than required */
+} attn_status;
+
+/*
+ * Prefill / full forward pass, bf16 output.
+ *   q   : device, bf16 [B, Nq, Hq, d], 16-byte aligned
+ *   k,v : device, bf16 [B, Nk, Hkv, d], 16-byte aligned
+ *   o   : device, bf16 [B, Nq, Hq, d], 16-byte aligned (written)
+ *   lse : device, f32 [B, Hq, Nq], 4-byte aligned, or NULL (not written)
+ *   B, Hq, Hkv, Nq, Nk >= 1; Hq % Hkv == 0; d in {64, 128}
+ *   scale : finite, > 0 (usually 1/sqrt(d))
+ *   causal : 0 or 1;  window_left : < 0 for none, else keys before the query
+ * Returns ATTN_OK or an attn_status; nothing is launched on error.
+ */
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+             int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+             int causal, int window_left, cudaStream_t stream);
+
+/* Same as attn_fwd, but o is float32 [B, Nq, Hq, d]. */
+int attn_fwd_f32o(const void* q, const void* k, const void* v, float* o, float* lse,
+                  int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+                  int causal, int window_left, cudaStream_t stream);
+
+/*
+ * Bytes of device workspace attn_decode needs for these sizes.
+ * num_splits = 0 picks the split count attn_decode would pick automatically.
+ * Returns 0 for invalid sizes.
+ */
+size_t attn_decode_workspace_bytes(int B, int Hq, int d, int num_splits, int Lmax);
+
+/*
+ * Single-query decode over a contiguous KV cache (split-KV + combine).
+ *   q        : device, bf16 [B, Hq, d]
+ *   k_cache  : device, bf16 [B, Lmax, Hkv, d]; v_cache likewise
+ *   o        : device, bf16 [B, Hq, d] (written)
+ *   lse      : device, f32 [B, Hq] or NULL
+ *   seqlens  : device, int32 [B] with 0 <= seqlens[b] <= Lmax, or NULL (= Lmax
+ *              for all). The query of sequence b sits at position
+ *              seqlens[b] - 1: its own K/V are already in the cache. A
+ *              sequence with seqlens[b] == 0 gets O = 0, LSE = -inf. Values
+ *              outside [0, Lmax] are clamped into that range on the device.
+ *   window_left : < 0 for none, else keys before the query's own position
+ *   num_splits  : key splits per (sequence, kv head); 0 = automatic
+ *   workspace   : device, >= attn_decode_workspace_bytes(...) bytes,
+ *                 256-byte aligned; contents on entry are ignored
+ * Returns ATTN_OK or an attn_status (ATTN_ERR_WORKSPACE if too small).
+ */
+int attn_decode(const void* q, const void* k_cache, const void* v_cache, void* o,
+                float* lse, const int* seqlens, int B, int Hq, int Hkv, int Lmax,
+                int d, float scale, int window_left, int num_splits,
+                void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Message for the last non-OK status returned on this host thread ("" if none). */
+const char* attn_last_error(void);
+
+/*
+ * Synchronises `stream`, then reads and clears the device status word that
+ * kernels set when a bounded wait gives up. Returns ATTN_OK, ATTN_ERR_TIMEOUT
+ * or ATTN_ERR_CUDA (a CUDA error surfaced by the synchronisation).
+ */
+int attn_device_status(cudaStream_t stream);
+
+/* Number of kernel launches this library has issued in this process. */
+unsigned long long attn_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_H_ */

@@ -1,0 +1,153 @@
+"""Host-side checks of the C ABI: the library loads, exports everything the
+header declares, and rejects bad arguments before touching the device.
+
+No test here launches a kernel: every call that reaches the library carries
+exactly one invalid argument, which the host-side validation catches first.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from exact_softmax_attention_03_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_expected_entry_points():
+    assert header_functions() == sorted([
+        "attn_fwd", "attn_fwd_f32o", "attn_decode_workspace_bytes", "attn_decode",
+        "attn_last_error", "attn_device_status", "attn_launch_count"])
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in header_functions():
+        assert hasattr(lib, name), name
+    assert sorted(_lib.SIGNATURES) == header_functions()
+
+
+def test_status_codes_match_header():
+    text = open(HEADER).read()
+    for name, val in re.findall(r"(ATTN_[A-Z_]+)\s*=\s*(\d+)", text):
+        assert getattr(_lib, name) == int(val)
+
+
+P = 0x100000          # a 16-byte-aligned non-null address that is never dereferenced
+
+
+def fwd_args(**over):
+    a = dict(q=P, k=P, v=P, o=P, lse=None, B=1, Hq=4, Hkv=2, Nq=128, Nk=128, d=128,
+             scale=0.125, causal=1, window_left=-1, stream=None)
+    a.update(over)
+    return [a[k] for k in ("q", "k", "v", "o", "lse", "B", "Hq", "Hkv", "Nq", "Nk", "d",
+                           "scale", "causal", "window_left", "stream")]
+
+
+BAD_FWD = [
+    (dict(q=None), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(o=None), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(B=0), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(Nk=0), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(Hq=6, Hkv=4), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(d=96), _lib.ATTN_ERR_UNSUPPORTED),
+    (dict(d=256), _lib.ATTN_ERR_UNSUPPORTED),
+    (dict(scale=0.0), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(causal=2), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(k=P + 8), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(o=P + 2), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(lse=P + 1), _lib.ATTN_ERR_INVALID_ARG),
+]
+
+
+@pytest.mark.parametrize("entry", ["attn_fwd", "attn_fwd_f32o"])
+@pytest.mark.parametrize("over,code", BAD_FWD)
+def test_fwd_rejects_bad_arguments_without_launch(lib, entry, over, code):
+    before = lib.attn_launch_count()
+    rc = getattr(lib, entry)(*fwd_args(**over))
+    assert rc == code, lib.attn_last_error()
+    assert lib.attn_last_error()
+    assert lib.attn_launch_count() == before
+
+
+def dec_args(**over):
+    a = dict(q=P, k=P, v=P, o=P, lse=None, seqlens=None, B=2, Hq=8, Hkv=2, Lmax=1000, d=128,
+             scale=0.1, window_left=-1, num_splits=0, ws=P, ws_bytes=1 << 30, stream=None)
+    a.update(over)
+    return [a[k] for k in ("q", "k", "v", "o", "lse", "seqlens", "B", "Hq", "Hkv", "Lmax", "d",
+                           "scale", "window_left", "num_splits", "ws", "ws_bytes", "stream")]
+
+
+BAD_DEC = [
+    (dict(q=None), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(Lmax=0), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(Hq=6, Hkv=4), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(d=80), _lib.ATTN_ERR_UNSUPPORTED),
+    (dict(scale=-1.0), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(num_splits=-1), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(v=P + 4), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(seqlens=P + 2), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(ws=None), _lib.ATTN_ERR_WORKSPACE),
+    (dict(ws_bytes=16), _lib.ATTN_ERR_WORKSPACE),
+    (dict(ws=P + 16), _lib.ATTN_ERR_INVALID_ARG),
+]
+
+
+@pytest.mark.parametrize("over,code", BAD_DEC)
+def test_decode_rejects_bad_arguments_without_launch(lib, over, code):
+    before = lib.attn_launch_count()
+    rc = lib.attn_decode(*dec_args(**over))
+    assert rc == code, lib.attn_last_error()
+    assert lib.attn_launch_count() == before
+
+
+def test_workspace_bytes(lib):
+    f = lib.attn_decode_workspace_bytes
+    assert f(0, 8, 128, 0, 100) == 0
+    assert f(2, 8, 96, 0, 100) == 0
+    assert f(2, 8, 128, -1, 100) == 0
+    one = f(2, 8, 128, 1, 1000)
+    # one split: B*Hq*d floats of partial output + B*Hq*2 floats of (max, sum), 256-byte rounded
+    assert one == ((2 * 8 * 128 * 4 + 255) // 256 * 256) + ((2 * 8 * 2 * 4 + 255) // 256 * 256)
+    assert f(2, 8, 128, 4, 1000) > one
+    assert f(64, 32, 128, 0, 8192) > 0
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_valid_call_without_a_device_reports_cuda_error(lib):
+    rc = lib.attn_fwd(*fwd_args())
+    assert rc == _lib.ATTN_ERR_CUDA
+    assert lib.attn_launch_count() == 0
+
+
+def test_binding_refuses_cpu_tensors():
+    import exact_softmax_attention_03_b200 as ea
+    q = torch.zeros(1, 8, 2, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        ea.attn_fwd(q, q, q)
+    with pytest.raises(ValueError, match="CUDA"):
+        ea.attn_decode(torch.zeros(1, 2, 64, dtype=torch.bfloat16), q, q)
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "libattn.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        _lib.load()

@@ -1,0 +1,133 @@
+"""GPU parity of attn_fwd / attn_fwd_f32o against the fp64 oracle.
+
+Small problems are compared element by element over every output; the full
+workload sizes (MHA 2K and 8K causal, GQA sliding window at 32K) run in the
+same launch configuration the bench times and are compared on sampled rows
+that the oracle computes one by one.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import attn_inputs as ai
+import oracle
+from parity import assert_close, cuda, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from exact_softmax_attention_03_b200 import build
+    build.build()
+
+
+def run_fwd(q, k, v, causal, wl, f32=False, scale=None, with_lse=True):
+    import exact_softmax_attention_03_b200 as ea
+    qg, kg, vg = cuda(q, k, v)
+    B, Nq, Hq, d = q.shape
+    lse = torch.full((B, Hq, Nq), 7.0, device="cuda") if with_lse else None
+    fn = ea.attn_fwd_f32o if f32 else ea.attn_fwd
+    o, _ = fn(qg, kg, vg, lse=lse, causal=causal, window_left=wl, scale=scale)
+    assert ea.attn_device_status() == 0
+    return o, lse
+
+
+def check_full(shape, causal, wl, f32=False, seed=ai.SEED_Q, scale=None):
+    B, Hq, Hkv, Nq, Nk, d = shape
+    q, k, v = ai.make_qkv(B, Hq, Hkv, Nq, Nk, d, seed)
+    o, lse = run_fwd(q, k, v, causal, wl, f32=f32, scale=scale)
+    O, L = oracle.oracle_attention(q, k, v, causal=causal, window_left=wl, scale=scale)
+    return assert_close(o, O, lse, L, what=(shape, causal, wl))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_tiny_workload_fp32_out(causal):
+    w = ai.TINY_CAUSAL if causal else ai.TINY
+    check_full((w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d), w.causal, w.window_left, f32=True)
+
+
+SHAPES = [
+    # (B, Hq, Hkv, Nq, Nk, d), causal, window_left
+    ((1, 2, 2, 1, 1, 128), True, -1),
+    ((1, 2, 2, 127, 127, 128), True, -1),
+    ((1, 2, 2, 129, 129, 128), False, -1),
+    ((2, 4, 4, 1000, 1000, 128), True, -1),
+    ((1, 2, 2, 100, 300, 128), True, -1),        # Nq < Nk: bottom-right alignment
+    ((1, 2, 2, 300, 100, 128), True, -1),        # Nq > Nk: leading rows see no key
+    ((1, 4, 1, 515, 515, 128), True, 0),         # MQA, window of one key
+    ((1, 4, 1, 515, 515, 128), True, 1),
+    ((1, 4, 1, 515, 515, 128), True, 127),
+    ((1, 4, 1, 515, 515, 128), True, 128),
+    ((1, 4, 1, 515, 515, 128), True, 129),
+    ((1, 8, 2, 384, 384, 128), True, 200),       # GQA, head pairs share K/V tiles
+    ((1, 6, 2, 300, 300, 64), True, -1),         # odd group size (3)
+    ((1, 4, 4, 257, 257, 64), False, 50),        # window without causal
+    ((2, 2, 1, 640, 640, 64), True, -1),
+    ((1, 1, 1, 2048, 2048, 128), False, -1),
+    ((1, 2, 2, 700, 1500, 128), False, 300),
+    ((1, 2, 2, 1, 4000, 128), True, -1),         # one query at the end of a long key set
+]
+
+
+@pytest.mark.parametrize("shape,causal,wl", SHAPES)
+def test_parity_shapes(shape, causal, wl):
+    check_full(shape, causal, wl)
+
+
+def test_parity_fp32_out_ragged():
+    check_full((1, 4, 2, 333, 333, 128), True, 100, f32=True)
+
+
+def test_custom_scale():
+    check_full((1, 2, 2, 200, 200, 128), True, -1, scale=0.3)
+
+
+def test_no_lse_pointer():
+    q, k, v = ai.make_qkv(1, 2, 2, 256, 256, 128)
+    o, _ = run_fwd(q, k, v, True, -1, with_lse=False)
+    O, _ = oracle.oracle_attention(q, k, v, causal=True)
+    assert_close(o, O)
+
+
+def test_fully_masked_rows_are_exact_zero_and_minus_inf():
+    q, k, v = ai.make_qkv(1, 2, 2, 300, 100, 128)
+    o, lse = run_fwd(q, k, v, True, -1)
+    assert (o[:, :200].float() == 0).all()
+    assert torch.isneginf(lse[:, :, :200]).all()
+    assert torch.isfinite(lse[:, :, 200:]).all()
+
+
+def test_deterministic_bitwise():
+    q, k, v = ai.make_qkv(2, 8, 2, 700, 700, 128)
+    o1, l1 = run_fwd(q, k, v, True, 300)
+    o2, l2 = run_fwd(q, k, v, True, 300)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_constant_v_gives_constant_output():
+    q, k, _ = ai.make_qkv(1, 4, 4, 500, 500, 128)
+    v = torch.full_like(k, 0.625)
+    o, _ = run_fwd(q, k, v, True, -1)
+    assert torch.allclose(o.float(), torch.full_like(o.float(), 0.625), atol=4e-3)
+
+
+FULL = [ai.MHA_2K, ai.MHA_8K, ai.GQA_SWA_32K]
+
+
+@pytest.mark.parametrize("w", FULL, ids=lambda w: w.name)
+def test_full_size_sampled_rows(w):
+    q, k, v = ai.make_for(w)
+    o, lse = run_fwd(q, k, v, w.causal, w.window_left)
+    assert torch.isfinite(o.float()).all()
+    assert torch.isfinite(lse).all()
+    g = torch.Generator().manual_seed(99)
+    for b, hq in [(0, 0), (w.B - 1, w.Hq - 1), (int(torch.randint(w.B, (1,), generator=g)),
+                                                int(torch.randint(w.Hq, (1,), generator=g)))]:
+        rows = sample_rows(w.Nq, 24, seed=b * 1000 + hq)
+        O, L = oracle.oracle_attention_rows(q, k, v, b, hq, rows, causal=w.causal,
+                                            window_left=w.window_left)
+        assert_close(o[b, rows, hq], O, lse[b, hq, rows], L, what=(w.name, b, hq))
