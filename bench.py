@@ -23,6 +23,7 @@ implementation of this path), one bounded per-head sample per step.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -42,8 +43,12 @@ from exact_softmax_attention_03_b200 import metrics  # noqa: E402
 
 METRIC = "attn fwd TFLOP/s (mask-adjusted) & % bf16 peak; decode KV-read GB/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ["exact_softmax_attention_03_b200/csrc/" + f for f in
-                  ("attn_api.cu", "sm100_ptx.cuh", "prefill_kernel.cuh", "decode_kernels.cuh")]
+KERNEL_SOURCES = {
+    "attn_fwd_kernel": ["exact_softmax_attention_03_b200/csrc/" + f
+                        for f in ("sm100_ptx.cuh", "prefill_kernel.cuh")],
+    "decode": ["exact_softmax_attention_03_b200/csrc/" + f
+               for f in ("sm100_ptx.cuh", "decode_kernels.cuh")],
+}
 
 
 def parse_args():
@@ -55,6 +60,10 @@ def parse_args():
     ap.add_argument("--workload", choices=["mha2k", "mha8k", "gqa32k"], default="mha2k",
                     help="prefill workload (default: the MHA causal prefill at N=2048)")
     ap.add_argument("--decode-splits", type=int, default=0)
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the prefill batch (profiling a smaller case only)")
+    ap.add_argument("--decode-batch", type=int, default=0,
+                    help="override the decode batch (profiling a smaller case only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -72,9 +81,10 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(kernel: str) -> str:
+    """Short hash of the device sources of one kernel family."""
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -85,7 +95,7 @@ def recorded_traffic(kernel: str, workload: str):
     path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
     if not os.path.exists(path):
         return None
-    want = kernel_source_hash()
+    want = kernel_source_hash(kernel)
     with open(path) as f:
         for line in f:
             parts = line.split()
@@ -327,6 +337,8 @@ def run_ours(args, world, rank, local):
     sampler = ClockSampler(torch.cuda.current_device() if world == 1 else local)
 
     w = PREFILL[args.workload]
+    if args.batch:
+        w = dataclasses.replace(w, B=args.batch, name=f"{w.name} [batch {args.batch}]")
     q_h, k_h, v_h = ai.make_for(w, seed=ai.SEED_Q + 17 * rank)
     q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
     o = torch.empty((w.B, w.Nq, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
@@ -350,6 +362,8 @@ def run_ours(args, world, rank, local):
 
     # decode leg
     dw = ai.GQA_DECODE
+    if args.decode_batch:
+        dw = dataclasses.replace(dw, B=args.decode_batch, name=f"{dw.name} [batch {args.decode_batch}]")
     qd_h, kc_h, vc_h = ai.make_decode(dw.B, dw.Hq, dw.Hkv, dw.Nk, dw.d, seed=ai.SEED_Q + 17 * rank)
     qd, kc, vc = qd_h.to(dev), kc_h.to(dev), vc_h.to(dev)
     od = torch.empty((dw.B, dw.Hq, dw.d), dtype=torch.bfloat16, device=dev)
@@ -436,7 +450,7 @@ def run_ours(args, world, rank, local):
         "gpu_launches": launches,
         "e2e": e2e,
         "cpu_baseline": cpu,
-        "kernel_sources": kernel_source_hash(),
+        "kernel_sources": {k: kernel_source_hash(k) for k in KERNEL_SOURCES},
     }
     print(json.dumps(line), flush=True)
 
