@@ -20,6 +20,7 @@ import torch
 from ._lib import AttnError, check, load  # noqa: F401
 
 __all__ = ["attn_fwd", "attn_fwd_f32o", "attn_decode", "attn_decode_workspace_bytes",
+           "attn_decode_noalloc",
            "attn_device_status", "attn_last_error", "attn_launch_count", "AttnError"]
 
 
@@ -121,6 +122,43 @@ def attn_decode(q, k_cache, v_cache, o=None, lse=None, seqlens=None, window_left
                              seqlens.data_ptr() if seqlens is not None else None,
                              B, Hq, Hkv, Lmax, d, float(scale), int(window_left), int(num_splits),
                              workspace.data_ptr(), ws_bytes, _stream_handle(stream)))
+    return o, lse
+
+
+def attn_decode_noalloc(q, k_cache, v_cache, o=None, lse=None, seqlens=None, window_left=-1,
+                        scale=None, num_splits=0, stream=None):
+    """Decode like :func:`attn_decode`, but the library keeps the partial results
+    in its own fixed device scratch, so no workspace is passed or allocated.
+
+    For callers that must not allocate device memory themselves (their host
+    program owns all device memory through its own pool, or an allocation's
+    possible device synchronisation is not acceptable on their path). ``o``
+    (and ``lse``, if wanted) must still be given, or ``o`` is allocated here by
+    torch for convenience. Calls on one device share the scratch: do not let
+    two of them overlap on the GPU. Sizes needing more than
+    ``ATTN_DECODE_NOALLOC_SCRATCH_BYTES`` of partials raise ``AttnError``.
+    """
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    _need(v_cache, "v_cache", torch.bfloat16, 4)
+    B, Hq, d = q.shape
+    _, Lmax, Hkv, _ = k_cache.shape
+    if k_cache.shape[0] != B or k_cache.shape[3] != d or v_cache.shape != k_cache.shape:
+        raise ValueError("caches must be [B, Lmax, Hkv, d] matching q")
+    if o is None:
+        o = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q.device)
+    _need(o, "o", torch.bfloat16, 3)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, 2)
+    if seqlens is not None:
+        _need(seqlens, "seqlens", torch.int32, 1)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    check(load().attn_decode_noalloc(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                                     o.data_ptr(), lse.data_ptr() if lse is not None else None,
+                                     seqlens.data_ptr() if seqlens is not None else None,
+                                     B, Hq, Hkv, Lmax, d, float(scale), int(window_left),
+                                     int(num_splits), _stream_handle(stream)))
     return o, lse
 
 

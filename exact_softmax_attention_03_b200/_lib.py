@@ -15,6 +15,9 @@ ATTN_ERR_CUDA = 3
 ATTN_ERR_TIMEOUT = 4
 ATTN_ERR_WORKSPACE = 5
 
+# Size of the fixed device scratch behind attn_decode_noalloc (include/attn.h).
+ATTN_DECODE_NOALLOC_SCRATCH_BYTES = 8 << 20
+
 STATUS_NAMES = {
     ATTN_OK: "ATTN_OK",
     ATTN_ERR_INVALID_ARG: "ATTN_ERR_INVALID_ARG",
@@ -35,6 +38,8 @@ SIGNATURES = {
     "attn_decode_workspace_bytes": (ctypes.c_size_t, [_i, _i, _i, _i, _i]),
     "attn_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _i, _vp,
                          ctypes.c_size_t, _vp]),
+    "attn_decode_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _i,
+                                 _vp]),
     "attn_last_error": (ctypes.c_char_p, []),
     "attn_device_status": (_i, [_vp]),
     "attn_launch_count": (ctypes.c_ulonglong, []),

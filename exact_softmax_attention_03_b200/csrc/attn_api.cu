@@ -226,9 +226,94 @@ void launch_decode_kernels(const attn::DecodeParams& p, cudaStream_t stream) {
   attn::decode_combine_kernel<D><<<(n + 3) / 4, 128, 0, stream>>>(p);
 }
 
+// ------------------------------------------------------ no-alloc decode --
+// Fixed scratch for attn_decode_noalloc: the library's own device memory, so
+// that callers which cannot allocate still get a split-KV decode. Host code
+// must not pass this symbol itself to a kernel (on the host it is only a
+// stand-in); it passes the device address looked up below.
+static __device__ __align__(256) unsigned char g_decode_noalloc_scratch[ATTN_DECODE_NOALLOC_SCRATCH_BYTES];
+
+// Device address of the scratch array for device `dev` (the current device),
+// looked up once per device and cached.
+int noalloc_scratch(int dev, void** out) {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  if (dev < 0 || dev >= 64) return fail(ATTN_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_decode_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return fail(ATTN_ERR_CUDA, "cudaGetSymbolAddress(decode scratch): %s", cudaGetErrorString(e));
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return ATTN_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+int attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, void* o,
+                        float* lse, const int* seqlens, int B, int Hq, int Hkv, int Lmax, int d,
+                        float scale, int window_left, int num_splits, cudaStream_t stream) {
+  if (!q || !k_cache || !v_cache || !o)
+    return fail(ATTN_ERR_INVALID_ARG, "q, k_cache, v_cache and o must be non-null");
+  if (B < 1 || Hq < 1 || Hkv < 1 || Lmax < 1)
+    return fail(ATTN_ERR_INVALID_ARG, "B, Hq, Hkv, Lmax must be >= 1");
+  if (Hq % Hkv != 0) return fail(ATTN_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
+  if (d != 64 && d != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim %d not in {64, 128}", d);
+  if (!finite_pos(scale)) return fail(ATTN_ERR_INVALID_ARG, "scale must be finite and > 0");
+  if (num_splits < 0) return fail(ATTN_ERR_INVALID_ARG, "num_splits must be >= 0");
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(o, 16))
+    return fail(ATTN_ERR_INVALID_ARG, "q, k_cache, v_cache, o must be 16-byte aligned");
+  if (lse && !aligned(lse, 4)) return fail(ATTN_ERR_INVALID_ARG, "lse must be 4-byte aligned");
+  if (seqlens && !aligned(seqlens, 4)) return fail(ATTN_ERR_INVALID_ARG, "seqlens must be 4-byte aligned");
+  if (static_cast<long long>(B) * Lmax > kMaxIndex || static_cast<long long>(B) * Hq > kMaxIndex)
+    return fail(ATTN_ERR_INVALID_ARG, "sizes too large");
+  const DecodeShape sh = decode_shape(B, Hq, d, num_splits, Lmax);
+  if (sh.total > ATTN_DECODE_NOALLOC_SCRATCH_BYTES)
+    return fail(ATTN_ERR_WORKSPACE,
+                "these sizes need %zu bytes of scratch (%d splits) but the fixed scratch holds %zu; "
+                "use attn_decode with a caller workspace or fewer splits",
+                sh.total, sh.S, static_cast<size_t>(ATTN_DECODE_NOALLOC_SCRATCH_BYTES));
+  int dev = 0;
+  int rc = check_device(&dev);
+  if (rc != ATTN_OK) return rc;
+  void* scratch = nullptr;
+  if ((rc = noalloc_scratch(dev, &scratch)) != ATTN_OK) return rc;
+
+  attn::DecodeParams p{};
+  p.q = static_cast<const uint16_t*>(q);
+  p.k = static_cast<const uint16_t*>(k_cache);
+  p.v = static_cast<const uint16_t*>(v_cache);
+  p.o = static_cast<uint16_t*>(o);
+  p.lse = lse;
+  p.seqlens = seqlens;
+  p.ws_acc = static_cast<float*>(scratch);
+  p.ws_ml = reinterpret_cast<float*>(static_cast<char*>(scratch) + sh.acc_bytes);
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Lmax = Lmax;
+  p.S = sh.S;
+  p.chunk = sh.chunk;
+  p.window_left = window_left < 0 ? -1 : window_left;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const int GT = decode_group_tile(Hq / Hkv);
+  if (d == 128) {
+    if (GT == 4) launch_decode_kernels<128, 4>(p, stream);
+    else if (GT == 2) launch_decode_kernels<128, 2>(p, stream);
+    else launch_decode_kernels<128, 1>(p, stream);
+  } else {
+    if (GT == 4) launch_decode_kernels<64, 4>(p, stream);
+    else if (GT == 2) launch_decode_kernels<64, 2>(p, stream);
+    else launch_decode_kernels<64, 1>(p, stream);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "attn_decode_noalloc launch: %s", cudaGetErrorString(e));
+  g_launches.fetch_add(2);
+  return ok();
+}
+
 
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
              int Hkv, int Nq, int Nk, int d, float scale, int causal, int window_left,

@@ -32,7 +32,8 @@
  *
  * Ownership. The caller allocates and owns every buffer (device memory),
  * including the decode workspace; the library never allocates or frees device
- * memory. All calls are asynchronous on `stream` (may be NULL = legacy default
+ * memory (the one exception is the fixed scratch array of
+ * attn_decode_noalloc, described there). All calls are asynchronous on `stream` (may be NULL = legacy default
  * stream) and never synchronise, except attn_device_status.
  *
  * Errors. Every entry point validates its arguments on the host first; on any
@@ -107,6 +108,37 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache, void* o
                 float* lse, const int* seqlens, int B, int Hq, int Hkv, int Lmax,
                 int d, float scale, int window_left, int num_splits,
                 void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Decode without a workspace argument, for callers that cannot allocate
+ * device memory. The pages have no counterpart to this; it exists for library
+ * users only. Typical callers: a host program that owns every byte of device
+ * memory through its own pool and forbids outside allocations, or a code path
+ * with a hard latency bound, where cudaMalloc (which may synchronise the
+ * device or fail under memory pressure) is not acceptable.
+ *
+ * Arguments, layouts and results are those of attn_decode, minus workspace
+ * and workspace_bytes. The partial results live instead in one fixed scratch
+ * array inside the library: ATTN_DECODE_NOALLOC_SCRATCH_BYTES bytes of device
+ * memory that every GPU which loads the library holds until the process exits.
+ * A call whose split count needs more scratch than that (see
+ * attn_decode_workspace_bytes) returns ATTN_ERR_WORKSPACE and launches
+ * nothing; use attn_decode with a caller buffer, or fewer splits, instead.
+ *
+ * The first call on each device (with that device current) looks up the
+ * scratch array's device address once; make that first call before any stream
+ * capture. The scratch array is shared by every call on a device and keeps
+ * the last call's contents; nothing in it needs to start at zero, because
+ * each call writes every word it later reads. Calls that may overlap on the
+ * GPU (for example on two streams without ordering) race on the scratch and
+ * must not be issued that way. This entry point calls no cudaMalloc, cudaFree
+ * or other allocating routine.
+ */
+#define ATTN_DECODE_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+int attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, void* o,
+                        float* lse, const int* seqlens, int B, int Hq, int Hkv, int Lmax,
+                        int d, float scale, int window_left, int num_splits,
+                        cudaStream_t stream);
 
 /* Message for the last non-OK status returned on this host thread ("" if none). */
 const char* attn_last_error(void);
