@@ -80,6 +80,12 @@ struct FwdParams {
 };
 
 constexpr int kFwdThreads = 384;
+// Every kPolyEvery-th pair of exponentials in an unmasked score tile is
+// computed on the FMA pipe instead of the MUFU unit.
+#ifndef ATTN_POLY_EVERY
+#define ATTN_POLY_EVERY 4
+#endif
+constexpr int kPolyEvery = ATTN_POLY_EVERY;
 
 struct TileInfo {
   int hq, row0, active;    // query head, first row, any row < Nq
@@ -248,19 +254,32 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
       for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
 
-      if (block_needs_mask(p, T, j)) {
+      const bool masked = block_needs_mask(p, T, j);
+      if (masked) {
+        // allowed keys of this row, relative to the block: [lo_rel, hi_rel]
         const int kb0 = j * 128;
+        int hi = p.Nk - 1;
+        if (p.causal) hi = min(hi, qpos);
+        int lo = 0;
+        if (p.window_left >= 0) lo = qpos - p.window_left;
+        const int lo_rel = lo - kb0, hi_rel = hi - kb0;
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const int key = kb0 + c;
-          const bool allowed = key < p.Nk && (!p.causal || key <= qpos) &&
-                               (p.window_left < 0 || key >= qpos - p.window_left);
-          if (!allowed) s[c] = -CUDART_INF_F;
-        }
+        for (int c = 0; c < 128; ++c)
+          if (c < lo_rel || c > hi_rel) s[c] = -CUDART_INF_F;
       }
-      float mb = s[0];
+      // row max: 8 independent chains of 3-input max
+      float mx[8];
 #pragma unroll
-      for (int c = 1; c < 128; ++c) mb = fmaxf(mb, s[c]);
+      for (int i = 0; i < 8; ++i) mx[i] = s[i];
+#pragma unroll
+      for (int c = 8; c < 120; c += 16) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx[i] = max3f(mx[i], s[c + i], s[c + 8 + i]);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[120 + i]);
+      const float mb = fmaxf(max3f(mx[0], mx[1], mx[2]),
+                             fmaxf(max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       // Lazy rescale: keep the old maximum while the new one exceeds it by at
       // most 8 in log2 units (P values stay <= 256); the final O / l is exact
       // whichever maximum was used.
@@ -272,15 +291,37 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         m = m_new;
       }
       const float mo = (m == -CUDART_INF_F) ? 0.f : m * c2;
-      float ls = 0.f;
+      // P = 2^(s * c2 - mo) on pairs; in unmasked tiles every kPolyEvery-th
+      // pair goes to the FMA-pipe polynomial to offload the MUFU unit.
+      const uint64_t C2 = f2_pack(c2, c2), NMO = f2_pack(-mo, -mo);
+      uint64_t lacc[4] = {0, 0, 0, 0};
       uint32_t pk[64];
+      if (masked) {
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float p0 = ex2_approx(fmaf(s[2 * c], c2, -mo));
-        const float p1 = ex2_approx(fmaf(s[2 * c + 1], c2, -mo));
-        ls += p0 + p1;
-        pk[c] = pack_bf16x2(p0, p1);
+        for (int c = 0; c < 64; ++c) {
+          const float2 x = f2_unpack(f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), C2, NMO));
+          const float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
+          lacc[c & 3] = f2_add(lacc[c & 3], f2_pack(p0, p1));
+          pk[c] = pack_bf16x2(p0, p1);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const uint64_t x = f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), C2, NMO);
+          uint64_t e;
+          if ((c % kPolyEvery) == kPolyEvery - 1) {
+            e = exp2_poly_f2(x);
+          } else {
+            const float2 xx = f2_unpack(x);
+            e = f2_pack(ex2_approx(xx.x), ex2_approx(xx.y));
+          }
+          lacc[c & 3] = f2_add(lacc[c & 3], e);
+          const float2 ee = f2_unpack(e);
+          pk[c] = pack_bf16x2(ee.x, ee.y);
+        }
       }
+      const float2 l01 = f2_unpack(f2_add(f2_add(lacc[0], lacc[1]), f2_add(lacc[2], lacc[3])));
+      const float ls = l01.x + l01.y;
       l = fmaf(l, alpha, ls);
       tmem_st32(tS, pk);
       tmem_st32(tS + 32, pk + 32);

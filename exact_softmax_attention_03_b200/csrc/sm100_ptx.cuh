@@ -58,12 +58,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return done != 0;
 }
 
-// Wait until the phase with the given parity has completed. Gives up after
-// kWaitLimitNs, or as soon as *abort (if not null) is set by another thread of
-// the CTA; on a timeout it sets *abort and the device status word. Returns
-// whether the phase completed.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
-  if (mbar_try_wait(bar, parity)) return true;
+// Slow path of mbar_wait (kept out of line so the fast path stays cheap).
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort) {
   const unsigned long long t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -76,6 +72,15 @@ __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile i
       }
     }
   }
+}
+
+// Wait until the phase with the given parity has completed. Gives up after
+// kWaitLimitNs, or as soon as *abort (if not null) is set by another thread of
+// the CTA; on a timeout it sets *abort and the device status word. Returns
+// whether the phase completed.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, abort);
 }
 
 // Named barrier over `count` threads (a warpgroup uses 128).
@@ -223,6 +228,61 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// ---- packed fp32 pairs (Blackwell f32x2 arithmetic) -------------------------
+
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 f2_unpack(uint64_t v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for a pair of floats on the FMA pipe (no MUFU): range reduction
+// x = j + f with j = round(x) (add/subtract 1.5 * 2^23), a cubic for 2^f on
+// [-0.5, 0.5], then j added to the exponent field. The cubic's coefficients
+// are a minimax fit of relative error (linear program on a dense grid; see
+// fit_exp2_poly.py next to this package): max relative error 7.5e-5, far below
+// the bf16 rounding of P. Inputs are clamped to >= -125 so the exponent stays
+// normal; callers use it only where x is finite (unmasked score tiles).
+__device__ __forceinline__ uint64_t exp2_poly_f2(uint64_t x) {
+  const float2 xc = f2_unpack(x);
+  x = f2_pack(fmaxf(xc.x, -125.f), fmaxf(xc.y, -125.f));
+  const uint64_t t = f2_add(x, f2_pack(12582912.f, 12582912.f));
+  const uint64_t r = f2_add(t, f2_pack(-12582912.f, -12582912.f));
+  const uint64_t f = f2_fma(r, f2_pack(-1.f, -1.f), x);
+  uint64_t q = f2_fma(f, f2_pack(0x1.c3f888p-5f, 0x1.c3f888p-5f), f2_pack(0x1.f0de1ep-3f, 0x1.f0de1ep-3f));
+  q = f2_fma(q, f, f2_pack(0x1.62f316p-1f, 0x1.62f316p-1f));
+  q = f2_fma(q, f, f2_pack(0x1.fff692p-1f, 0x1.fff692p-1f));
+  const float2 qq = f2_unpack(q), tt = f2_unpack(t);
+  const uint32_t e0 = __float_as_uint(qq.x) + (__float_as_uint(tt.x) << 23);
+  const uint32_t e1 = __float_as_uint(qq.y) + (__float_as_uint(tt.y) << 23);
+  return f2_pack(__uint_as_float(e0), __uint_as_float(e1));
 }
 
 // 16-byte streaming load that bypasses L1 allocation (read-only data).
