@@ -10,6 +10,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 
 #include "../../include/attn.h"
@@ -56,6 +57,21 @@ int check_device(int* dev_out) {
   if (dev >= 0 && dev < 64) cache[dev].store(good ? 1 : 2);
   if (!good) return fail(ATTN_ERR_UNSUPPORTED, "device %d is sm_%d%d, need sm_100", dev, major, minor);
   *dev_out = dev;
+  return ATTN_OK;
+}
+
+// Number of SMs of device `dev`, cached per device ordinal.
+int sm_count(int dev, int* out) {
+  static std::atomic<int> cache[64];
+  if (dev >= 0 && dev < 64 && cache[dev].load() > 0) {
+    *out = cache[dev].load();
+    return ATTN_OK;
+  }
+  int n = 0;
+  cudaError_t e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess || n <= 0) return fail(ATTN_ERR_CUDA, "SM count: %s", cudaGetErrorString(e));
+  if (dev >= 0 && dev < 64) cache[dev].store(n);
+  *out = n;
   return ATTN_OK;
 }
 
@@ -141,8 +157,12 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     p.n_units = (p.n_qblk + 1) / 2;
     p.n_bh = B * Hq;
   }
-  const long long grid = static_cast<long long>(p.n_units) * p.n_bh;
-  if (grid > kMaxIndex) return fail(ATTN_ERR_INVALID_ARG, "problem too large for one launch");
+  const long long items = static_cast<long long>(p.n_units) * p.n_bh;
+  if (items > kMaxIndex) return fail(ATTN_ERR_INVALID_ARG, "problem too large for one launch");
+  p.n_items = static_cast<int>(items);
+  int sms = 0;
+  if ((rc = sm_count(dev, &sms)) != ATTN_OK) return rc;
+  const long long grid = std::min<long long>(items, sms);   // persistent: one CTA per SM
 
   static std::atomic<unsigned long long> attr_set{0};   // per-device bit
   const unsigned long long bit = 1ull << (dev & 63);

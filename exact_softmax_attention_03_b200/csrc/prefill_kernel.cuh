@@ -6,7 +6,12 @@
 // the accumulator when the maximum moves, divide by the sum at the end. The
 // score tile never leaves the SM: it lives in tensor memory (TMEM).
 //
-// One CTA (384 threads) owns two 128-row query tiles that share every K/V tile:
+// The kernel is persistent: one CTA (384 threads) per SM walks a static list
+// of work items (longest causal rows first, boustrophedon over the CTAs). The
+// K/V ring, the barrier phases and the Q buffers carry over from item to item,
+// so the next item's loads and first Q.K^T overlap the current item's tail
+// and epilogue. A work item is two 128-row query tiles that share every K/V
+// tile:
 //   * two heads of one K/V group at the same rows when Hq / Hkv is even
 //     (the grouped-query map of "Chapter 3: MHA Limitations, MQA, GQA, and
 //     FlashAttention", section 3.3, so each K/V tile is loaded once for both),
@@ -47,15 +52,17 @@ struct FwdLayout {
   static constexpr int OFF_V = OFF_K + STAGES * TILE;
   static constexpr int OFF_BAR = OFF_V + STAGES * TILE;
   // barrier indices
-  static constexpr int B_Q = 0;
-  static constexpr int B_KF = 1;                        // + stage
+  static constexpr int B_Q = 0;                         // Q tiles loaded
+  static constexpr int B_QE = 1;                        // Q tiles free (all Q.K^T done)
+  static constexpr int B_KF = 2;                        // + stage
   static constexpr int B_KE = B_KF + STAGES;
   static constexpr int B_VF = B_KE + STAGES;
   static constexpr int B_VE = B_VF + STAGES;
   static constexpr int B_SF = B_VE + STAGES;            // + tile
   static constexpr int B_PF = B_SF + 2;
-  static constexpr int B_OD = B_PF + 2;
-  static constexpr int B_DRAIN = B_OD + 2;
+  static constexpr int B_OD = B_PF + 2;                 // P.V done, + tile
+  static constexpr int B_OE = B_OD + 2;                 // O read by the epilogue, + tile
+  static constexpr int B_DRAIN = B_OE + 2;
   static constexpr int NBAR = B_DRAIN + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // [0] TMEM base, [1] abort flag
   static constexpr int BYTES = OFF_MISC + 16;
@@ -77,6 +84,7 @@ struct FwdParams {
   int n_qblk;              // ceil(Nq / 128)
   int n_units;             // row units per (b, head-or-pair)
   int n_bh;                // number of (b, head-or-pair) combinations
+  int n_items;             // n_units * n_bh
 };
 
 constexpr int kFwdThreads = 384;
@@ -142,6 +150,62 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint3
   }
 }
 
+// One work item: a (batch, head-or-head-pair, row unit) and its two tiles.
+struct WorkItem {
+  int b, hkv;
+  TileInfo tile[2];
+  int ubhi, U;             // key blocks visited: ubhi-1 down to ubhi-U
+};
+
+__device__ __forceinline__ void decode_item(const FwdParams& p, int item, WorkItem& w) {
+  const int unit = p.n_units - 1 - item / p.n_bh;        // longest rows first
+  const int bh = item % p.n_bh;
+  if (p.pair_heads) {
+    const int G = p.Hq / p.Hkv;
+    const int pairs = G / 2;
+    w.b = bh / (p.Hkv * pairs);
+    const int rem = bh % (p.Hkv * pairs);
+    w.hkv = rem / pairs;
+    const int pr = rem % pairs;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      w.tile[t].hq = w.hkv * G + 2 * pr + t;
+      w.tile[t].row0 = unit * 128;
+    }
+  } else {
+    w.b = bh / p.Hq;
+    const int hq = bh % p.Hq;
+    w.hkv = hq / (p.Hq / p.Hkv);
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      w.tile[t].hq = hq;
+      w.tile[t].row0 = (2 * unit + t) * 128;
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    w.tile[t].active = w.tile[t].row0 < p.Nq;
+    tile_range(p, w.tile[t]);
+  }
+  const bool ne0 = w.tile[0].bhi > w.tile[0].blo, ne1 = w.tile[1].bhi > w.tile[1].blo;
+  int ublo = 0, ubhi = 0;
+  if (ne0 || ne1) {
+    ublo = ne0 ? (ne1 ? min(w.tile[0].blo, w.tile[1].blo) : w.tile[0].blo) : w.tile[1].blo;
+    ubhi = ne0 ? (ne1 ? max(w.tile[0].bhi, w.tile[1].bhi) : w.tile[0].bhi) : w.tile[1].bhi;
+  }
+  w.ubhi = ubhi;
+  w.U = ubhi - ublo;
+}
+
+// k-th work item of this CTA in a boustrophedon order over the items sorted
+// longest first (close to a longest-processing-time schedule); -1 when done.
+__device__ __forceinline__ int item_of(const FwdParams& p, int k) {
+  const int G = int(gridDim.x);
+  const int c = (k & 1) ? (G - 1 - int(blockIdx.x)) : int(blockIdx.x);
+  const long long i = static_cast<long long>(k) * G + c;
+  return i < p.n_items ? int(i) : -1;
+}
+
 template <int D, bool F32OUT>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -158,49 +222,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work item -----------------------------------------------------------
-  const int unit = p.n_units - 1 - int(blockIdx.x) / p.n_bh;   // longest rows first
-  const int bh = int(blockIdx.x) % p.n_bh;
-  int b, hkv;
-  TileInfo tile[2];
-  if (p.pair_heads) {
-    const int G = p.Hq / p.Hkv;
-    const int pairs = G / 2;
-    b = bh / (p.Hkv * pairs);
-    const int rem = bh % (p.Hkv * pairs);
-    hkv = rem / pairs;
-    const int pr = rem % pairs;
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      tile[t].hq = hkv * G + 2 * pr + t;
-      tile[t].row0 = unit * 128;
-    }
-  } else {
-    b = bh / p.Hq;
-    const int hq = bh % p.Hq;
-    hkv = hq / (p.Hq / p.Hkv);
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      tile[t].hq = hq;
-      tile[t].row0 = (2 * unit + t) * 128;
-    }
-  }
-#pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    tile[t].active = tile[t].row0 < p.Nq;
-    tile_range(p, tile[t]);
-  }
-  const bool ne0 = tile[0].bhi > tile[0].blo, ne1 = tile[1].bhi > tile[1].blo;
-  int ublo = 0, ubhi = 0;
-  if (ne0 || ne1) {
-    ublo = ne0 ? (ne1 ? min(tile[0].blo, tile[1].blo) : tile[0].blo) : tile[1].blo;
-    ubhi = ne0 ? (ne1 ? max(tile[0].bhi, tile[1].bhi) : tile[0].bhi) : tile[1].bhi;
-  }
-  const int U = ubhi - ublo;              // key blocks visited, in descending order
-
   // ---- setup ---------------------------------------------------------------
   if (threadIdx.x == 0) {
     mbar_init(bar(L::B_Q), 1);
+    mbar_init(bar(L::B_QE), 1);
     for (int s = 0; s < L::STAGES; ++s) {
       mbar_init(bar(L::B_KF + s), 1);
       mbar_init(bar(L::B_KE + s), 1);
@@ -211,6 +236,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       mbar_init(bar(L::B_SF + t), 1);
       mbar_init(bar(L::B_PF + t), 128);
       mbar_init(bar(L::B_OD + t), 1);
+      mbar_init(bar(L::B_OE + t), 128);
     }
     mbar_init(bar(L::B_DRAIN), 1);
     *abort_flag = 0;
@@ -228,225 +254,258 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   if (warp < 8) {
     // ======================= softmax warpgroups ==============================
     const int t = warp >> 2;
-    const TileInfo& T = tile[t];
     const int row = int(threadIdx.x) - 128 * t;
     const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_off + (t ? L::COL_S1 : L::COL_S0);
     const uint32_t tO = tmem + lane_off + (t ? L::COL_O1 : L::COL_O0);
-    const int r = T.row0 + row;
-    const int qpos = r + p.Nk - p.Nq;
     const float c2 = p.scale_log2;
-    float m = -CUDART_INF_F;                // running max (raw score units)
-    float l = 0.f;                          // running sum of exp2((s - m) * c2)
-    int count = 0;
+    int count = 0;                          // S tiles processed so far (all items)
     bool ok = true;
-    for (int j = T.bhi - 1; j >= T.blo; --j) {
-      bool w = mbar_wait(bar(L::B_SF + t), uint32_t(count & 1), abort_flag);
-      if (w && count > 0) w = mbar_wait(bar(L::B_OD + t), uint32_t((count - 1) & 1), abort_flag);
-      if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
-      tc_fence_after();
+    for (int k = 0; ok; ++k) {
+      const int item = item_of(p, k);
+      if (item < 0) break;
+      WorkItem w;
+      decode_item(p, item, w);
+      const TileInfo& T = w.tile[t];
+      if (!T.active) continue;
+      const int r = T.row0 + row;
+      const int qpos = r + p.Nk - p.Nq;
+      float m = -CUDART_INF_F;              // running max (raw score units)
+      float l = 0.f;                        // running sum of exp2((s - m) * c2)
+      int n_in_item = 0;
+      for (int j = T.bhi - 1; j >= T.blo; --j) {
+        bool wt = mbar_wait(bar(L::B_SF + t), uint32_t(count & 1), abort_flag);
+        // the previous P.V of this item must be done before P is overwritten
+        // and before O is rescaled (at an item's first tile it was waited for
+        // in the previous epilogue)
+        if (wt && n_in_item > 0)
+          wt = mbar_wait(bar(L::B_OD + t), uint32_t((count - 1) & 1), abort_flag);
+        if (!__all_sync(0xffffffffu, wt)) { ok = false; break; }
+        tc_fence_after();
 
-      uint32_t sr[128];
+        uint32_t sr[128];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, sr + 32 * c);
-      tmem_wait_ld();
-      float s[128];
+        for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, sr + 32 * c);
+        tmem_wait_ld();
+        float s[128];
 #pragma unroll
-      for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
+        for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
 
-      const bool masked = block_needs_mask(p, T, j);
-      if (masked) {
-        // allowed keys of this row, relative to the block: [lo_rel, hi_rel]
-        const int kb0 = j * 128;
-        int hi = p.Nk - 1;
-        if (p.causal) hi = min(hi, qpos);
-        int lo = 0;
-        if (p.window_left >= 0) lo = qpos - p.window_left;
-        const int lo_rel = lo - kb0, hi_rel = hi - kb0;
+        const bool masked = block_needs_mask(p, T, j);
+        if (masked) {
+          // allowed keys of this row, relative to the block: [lo_rel, hi_rel]
+          const int kb0 = j * 128;
+          int hi = p.Nk - 1;
+          if (p.causal) hi = min(hi, qpos);
+          int lo = 0;
+          if (p.window_left >= 0) lo = qpos - p.window_left;
+          const int lo_rel = lo - kb0, hi_rel = hi - kb0;
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c < lo_rel || c > hi_rel) s[c] = -CUDART_INF_F;
-      }
-      // row max: 8 independent chains of 3-input max
-      float mx[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = s[i];
-#pragma unroll
-      for (int c = 8; c < 120; c += 16) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) mx[i] = max3f(mx[i], s[c + i], s[c + 8 + i]);
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[120 + i]);
-      const float mb = fmaxf(max3f(mx[0], mx[1], mx[2]),
-                             fmaxf(max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-      // Lazy rescale: keep the old maximum while the new one exceeds it by at
-      // most 8 in log2 units (P values stay <= 256); the final O / l is exact
-      // whichever maximum was used.
-      const float m_new = fmaxf(m, mb);
-      const bool rescale = (m_new - m) * c2 > 8.0f;       // false when both are -inf
-      float alpha = 1.f;
-      if (rescale) {
-        alpha = ex2_approx((m - m_new) * c2);              // 0 when m was -inf
-        m = m_new;
-      }
-      const float mo = (m == -CUDART_INF_F) ? 0.f : m * c2;
-      // P = 2^(s * c2 - mo) on pairs; in unmasked tiles every kPolyEvery-th
-      // pair goes to the FMA-pipe polynomial to offload the MUFU unit.
-      const uint64_t C2 = f2_pack(c2, c2), NMO = f2_pack(-mo, -mo);
-      uint64_t lacc[4] = {0, 0, 0, 0};
-      uint32_t pk[64];
-      if (masked) {
-#pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float2 x = f2_unpack(f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), C2, NMO));
-          const float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
-          lacc[c & 3] = f2_add(lacc[c & 3], f2_pack(p0, p1));
-          pk[c] = pack_bf16x2(p0, p1);
+          for (int c = 0; c < 128; ++c)
+            if (c < lo_rel || c > hi_rel) s[c] = -CUDART_INF_F;
         }
-      } else {
+        // row max: 8 independent chains of 3-input max
+        float mx[8];
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const uint64_t x = f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), C2, NMO);
-          uint64_t e;
-          if ((c % kPolyEvery) == kPolyEvery - 1) {
-            e = exp2_poly_f2(x);
-          } else {
-            const float2 xx = f2_unpack(x);
-            e = f2_pack(ex2_approx(xx.x), ex2_approx(xx.y));
+        for (int i = 0; i < 8; ++i) mx[i] = s[i];
+#pragma unroll
+        for (int c = 8; c < 120; c += 16) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mx[i] = max3f(mx[i], s[c + i], s[c + 8 + i]);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[120 + i]);
+        const float mb = fmaxf(max3f(mx[0], mx[1], mx[2]),
+                               fmaxf(max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        // Lazy rescale: keep the old maximum while the new one exceeds it by at
+        // most 8 in log2 units (P values stay <= 256); the final O / l is exact
+        // whichever maximum was used.
+        const float m_new = fmaxf(m, mb);
+        const bool rescale = (m_new - m) * c2 > 8.0f;     // false when both are -inf
+        float alpha = 1.f;
+        if (rescale) {
+          alpha = ex2_approx((m - m_new) * c2);            // 0 when m was -inf
+          m = m_new;
+        }
+        const float mo = (m == -CUDART_INF_F) ? 0.f : m * c2;
+        // P = 2^(s * c2 - mo) on pairs; in unmasked tiles every kPolyEvery-th
+        // pair goes to the FMA-pipe polynomial to offload the MUFU unit.
+        const uint64_t C2 = f2_pack(c2, c2), NMO = f2_pack(-mo, -mo);
+        uint64_t lacc[4] = {0, 0, 0, 0};
+        uint32_t pk[64];
+        if (masked) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            const float2 x = f2_unpack(f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), C2, NMO));
+            const float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
+            lacc[c & 3] = f2_add(lacc[c & 3], f2_pack(p0, p1));
+            pk[c] = pack_bf16x2(p0, p1);
           }
-          lacc[c & 3] = f2_add(lacc[c & 3], e);
-          const float2 ee = f2_unpack(e);
-          pk[c] = pack_bf16x2(ee.x, ee.y);
-        }
-      }
-      const float2 l01 = f2_unpack(f2_add(f2_add(lacc[0], lacc[1]), f2_add(lacc[2], lacc[3])));
-      const float ls = l01.x + l01.y;
-      l = fmaf(l, alpha, ls);
-      tmem_st32(tS, pk);
-      tmem_st32(tS + 32, pk + 32);
-
-      if (count > 0 && __any_sync(0xffffffffu, rescale)) {
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + 32 * c, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(tO + 32 * c, o);
-        }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(L::B_PF + t));
-      ++count;
-    }
-
-    // ---- epilogue: O / l and LSE -------------------------------------------
-    if (T.active) {
-      bool have = ok && count > 0;
-      if (have) have = mbar_wait(bar(L::B_OD + t), uint32_t((count - 1) & 1), abort_flag);
-      have = __all_sync(0xffffffffu, have);
-      if (have) tc_fence_after();
-      const bool store = r < p.Nq;
-      const float inv = (l > 0.f) ? 1.f / l : 0.f;
-      const size_t obase = ((size_t(b) * p.Nq + r) * p.Hq + T.hq) * D;
-#pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        if (have) {
-          tmem_ld32(tO + 32 * c, o);
-          tmem_wait_ld();
         } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = 0u;
-        }
-        if (store) {
-          if constexpr (F32OUT) {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + obase + 32 * c);
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-              dst[e] = make_float4(__uint_as_float(o[4 * e]) * inv, __uint_as_float(o[4 * e + 1]) * inv,
-                                   __uint_as_float(o[4 * e + 2]) * inv, __uint_as_float(o[4 * e + 3]) * inv);
-          } else {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) + obase + 32 * c);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              uint4 w;
-              w.x = pack_bf16x2(__uint_as_float(o[8 * e + 0]) * inv, __uint_as_float(o[8 * e + 1]) * inv);
-              w.y = pack_bf16x2(__uint_as_float(o[8 * e + 2]) * inv, __uint_as_float(o[8 * e + 3]) * inv);
-              w.z = pack_bf16x2(__uint_as_float(o[8 * e + 4]) * inv, __uint_as_float(o[8 * e + 5]) * inv);
-              w.w = pack_bf16x2(__uint_as_float(o[8 * e + 6]) * inv, __uint_as_float(o[8 * e + 7]) * inv);
-              dst[e] = w;
+          for (int c = 0; c < 64; ++c) {
+            const uint64_t x = f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), C2, NMO);
+            uint64_t e;
+            if ((c % kPolyEvery) == kPolyEvery - 1) {
+              e = exp2_poly_f2(x);
+            } else {
+              const float2 xx = f2_unpack(x);
+              e = f2_pack(ex2_approx(xx.x), ex2_approx(xx.y));
             }
+            lacc[c & 3] = f2_add(lacc[c & 3], e);
+            const float2 ee = f2_unpack(e);
+            pk[c] = pack_bf16x2(ee.x, ee.y);
           }
         }
+        const float2 l01 = f2_unpack(f2_add(f2_add(lacc[0], lacc[1]), f2_add(lacc[2], lacc[3])));
+        l = fmaf(l, alpha, l01.x + l01.y);
+        tmem_st32(tS, pk);
+        tmem_st32(tS + 32, pk + 32);
+
+        if (n_in_item > 0 && __any_sync(0xffffffffu, rescale)) {
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO + 32 * c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(tO + 32 * c, o);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(L::B_PF + t));
+        ++count;
+        ++n_in_item;
       }
-      if (store && p.lse != nullptr) {
-        p.lse[(size_t(b) * p.Hq + T.hq) * p.Nq + r] =
-            (l > 0.f) ? fmaf(m, p.scale, __log2f(l) * 0.6931471805599453f) : -CUDART_INF_F;
+      if (!ok) break;
+
+      // ---- epilogue: O / l and LSE -----------------------------------------
+      bool have = n_in_item > 0;
+      if (have) {
+        const bool wt = mbar_wait(bar(L::B_OD + t), uint32_t((count - 1) & 1), abort_flag);
+        if (!__all_sync(0xffffffffu, wt)) { ok = false; break; }
+        tc_fence_after();
+      }
+      uint32_t o[D];
+      if (have) {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) tmem_ld32(tO + 32 * c, o + 32 * c);
+        tmem_wait_ld();
+        // O of this tile has been read: the next item's first P.V may overwrite it
+        tc_fence_before();
+        mbar_arrive(bar(L::B_OE + t));
+      } else {
+#pragma unroll
+        for (int e = 0; e < D; ++e) o[e] = 0u;
+      }
+      if (r < p.Nq) {
+        const float inv = (l > 0.f) ? 1.f / l : 0.f;
+        const size_t obase = ((size_t(w.b) * p.Nq + r) * p.Hq + T.hq) * D;
+        if constexpr (F32OUT) {
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + obase);
+#pragma unroll
+          for (int e = 0; e < D / 4; ++e)
+            dst[e] = make_float4(__uint_as_float(o[4 * e]) * inv, __uint_as_float(o[4 * e + 1]) * inv,
+                                 __uint_as_float(o[4 * e + 2]) * inv, __uint_as_float(o[4 * e + 3]) * inv);
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) + obase);
+#pragma unroll
+          for (int e = 0; e < D / 8; ++e) {
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(o[8 * e + 0]) * inv, __uint_as_float(o[8 * e + 1]) * inv);
+            v.y = pack_bf16x2(__uint_as_float(o[8 * e + 2]) * inv, __uint_as_float(o[8 * e + 3]) * inv);
+            v.z = pack_bf16x2(__uint_as_float(o[8 * e + 4]) * inv, __uint_as_float(o[8 * e + 5]) * inv);
+            v.w = pack_bf16x2(__uint_as_float(o[8 * e + 6]) * inv, __uint_as_float(o[8 * e + 7]) * inv);
+            dst[e] = v;
+          }
+        }
+        if (p.lse != nullptr)
+          p.lse[(size_t(w.b) * p.Hq + T.hq) * p.Nq + r] =
+              (l > 0.f) ? fmaf(m, p.scale, __log2f(l) * 0.6931471805599453f) : -CUDART_INF_F;
       }
     }
   } else if (warp == 8) {
     // ======================= tensor-core issuer ==============================
-    if (lane == 0 && U > 0) {
+    if (lane == 0) {
       const uint32_t q0 = sb + L::OFF_Q, q1 = sb + L::OFF_Q + L::TILE;
       const uint32_t dS0 = tmem + L::COL_S0, dS1 = tmem + L::COL_S1;
       const uint32_t dO0 = tmem + L::COL_O0, dO1 = tmem + L::COL_O1;
-      int pv0 = 0, pv1 = 0;                 // P·V products issued per tile
-      int prev_j = -1, prev_slot = 0;
-      bool alive = mbar_wait(bar(L::B_Q), 0, abort_flag);
-      if (alive) tc_fence_after();
-      for (int it = 0; alive && it < U; ++it) {
-        const int j = ubhi - 1 - it;
-        const int slot = it % L::STAGES;
-        const uint32_t ph = uint32_t(it / L::STAGES) & 1u;
-        if (!(alive = mbar_wait(bar(L::B_KF + slot), ph, abort_flag))) break;
+      int pv0 = 0, pv1 = 0;                 // P.V products issued per tile (all items)
+      int done0 = 0, done1 = 0;             // items in which each tile had work
+      int kv = 0, qi = 0;                   // K/V ring position, items with a Q load
+      bool alive = true;
+      for (int k = 0; alive; ++k) {
+        const int item = item_of(p, k);
+        if (item < 0) break;
+        WorkItem w;
+        decode_item(p, item, w);
+        if (w.U == 0) continue;
+        if (!(alive = mbar_wait(bar(L::B_Q), uint32_t(qi & 1), abort_flag))) break;
         tc_fence_after();
-        const uint32_t ks = sb + L::OFF_K + slot * L::TILE;
-        if (tile_has(tile[0], j)) {
-          issue_qk<D>(dS0, q0, ks);
-          tc_commit(bar(L::B_SF + 0));
-        }
-        if (it > 0) {
-          if (tile_has(tile[1], prev_j)) {
-            if (!(alive = mbar_wait(bar(L::B_PF + 1), uint32_t(pv1 & 1), abort_flag))) break;
-            tc_fence_after();
-            issue_pv<D>(dO1, dS1, sb + L::OFF_V + prev_slot * L::TILE, pv1 > 0);
-            tc_commit(bar(L::B_OD + 1));
-            ++pv1;
-          }
-          tc_commit(bar(L::B_VE + prev_slot));
-        }
-        if (tile_has(tile[1], j)) {
-          issue_qk<D>(dS1, q1, ks);
-          tc_commit(bar(L::B_SF + 1));
-        }
-        tc_commit(bar(L::B_KE + slot));
-        if (!(alive = mbar_wait(bar(L::B_VF + slot), ph, abort_flag))) break;
-        tc_fence_after();
-        if (tile_has(tile[0], j)) {
-          if (!(alive = mbar_wait(bar(L::B_PF + 0), uint32_t(pv0 & 1), abort_flag))) break;
+        bool first0 = true, first1 = true;
+        int prev_j = -1, prev_slot = 0;
+        for (int it = 0; it < w.U; ++it, ++kv) {
+          const int j = w.ubhi - 1 - it;
+          const int slot = kv % L::STAGES;
+          const uint32_t ph = uint32_t(kv / L::STAGES) & 1u;
+          if (!(alive = mbar_wait(bar(L::B_KF + slot), ph, abort_flag))) break;
           tc_fence_after();
-          issue_pv<D>(dO0, dS0, sb + L::OFF_V + slot * L::TILE, pv0 > 0);
-          tc_commit(bar(L::B_OD + 0));
-          ++pv0;
-        }
-        prev_j = j;
-        prev_slot = slot;
-      }
-      if (alive && prev_j >= 0) {
-        if (tile_has(tile[1], prev_j)) {
-          alive = mbar_wait(bar(L::B_PF + 1), uint32_t(pv1 & 1), abort_flag);
-          if (alive) {
-            tc_fence_after();
-            issue_pv<D>(dO1, dS1, sb + L::OFF_V + prev_slot * L::TILE, pv1 > 0);
-            tc_commit(bar(L::B_OD + 1));
-            ++pv1;
+          const uint32_t ks = sb + L::OFF_K + slot * L::TILE;
+          if (tile_has(w.tile[0], j)) {
+            issue_qk<D>(dS0, q0, ks);
+            tc_commit(bar(L::B_SF + 0));
           }
+          if (it > 0) {
+            if (tile_has(w.tile[1], prev_j)) {
+              if (!(alive = mbar_wait(bar(L::B_PF + 1), uint32_t(pv1 & 1), abort_flag))) break;
+              if (first1 && done1 > 0 &&
+                  !(alive = mbar_wait(bar(L::B_OE + 1), uint32_t((done1 - 1) & 1), abort_flag))) break;
+              tc_fence_after();
+              issue_pv<D>(dO1, dS1, sb + L::OFF_V + prev_slot * L::TILE, !first1);
+              tc_commit(bar(L::B_OD + 1));
+              ++pv1;
+              first1 = false;
+            }
+            tc_commit(bar(L::B_VE + prev_slot));
+          }
+          if (tile_has(w.tile[1], j)) {
+            issue_qk<D>(dS1, q1, ks);
+            tc_commit(bar(L::B_SF + 1));
+          }
+          tc_commit(bar(L::B_KE + slot));
+          if (it == w.U - 1) tc_commit(bar(L::B_QE));     // every Q.K^T of this item issued
+          if (!(alive = mbar_wait(bar(L::B_VF + slot), ph, abort_flag))) break;
+          tc_fence_after();
+          if (tile_has(w.tile[0], j)) {
+            if (!(alive = mbar_wait(bar(L::B_PF + 0), uint32_t(pv0 & 1), abort_flag))) break;
+            if (first0 && done0 > 0 &&
+                !(alive = mbar_wait(bar(L::B_OE + 0), uint32_t((done0 - 1) & 1), abort_flag))) break;
+            tc_fence_after();
+            issue_pv<D>(dO0, dS0, sb + L::OFF_V + slot * L::TILE, !first0);
+            tc_commit(bar(L::B_OD + 0));
+            ++pv0;
+            first0 = false;
+          }
+          prev_j = j;
+          prev_slot = slot;
+        }
+        if (!alive) break;
+        if (tile_has(w.tile[1], prev_j)) {
+          if (!(alive = mbar_wait(bar(L::B_PF + 1), uint32_t(pv1 & 1), abort_flag))) break;
+          if (first1 && done1 > 0 &&
+              !(alive = mbar_wait(bar(L::B_OE + 1), uint32_t((done1 - 1) & 1), abort_flag))) break;
+          tc_fence_after();
+          issue_pv<D>(dO1, dS1, sb + L::OFF_V + prev_slot * L::TILE, !first1);
+          tc_commit(bar(L::B_OD + 1));
+          ++pv1;
+          first1 = false;
         }
         tc_commit(bar(L::B_VE + prev_slot));
+        if (!first0) ++done0;
+        if (!first1) ++done1;
+        ++qi;
       }
       // drain: every issued tensor-core operation completes before teardown
       tc_commit(bar(L::B_DRAIN));
@@ -455,37 +514,49 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     __syncwarp();
   } else if (warp == 9) {
     // ======================= TMA producer ====================================
-    if (lane == 0 && U > 0) {
+    if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(bar(L::B_Q), 2 * L::TILE);
-#pragma unroll
-      for (int t = 0; t < 2; ++t)
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_4d(sb + L::OFF_Q + t * L::TILE + c * L::HALF, &tmQ, bar(L::B_Q), c * 64,
-                      tile[t].hq, tile[t].row0, b);
+      int kv = 0, qi = 0;                   // same counters as the issuer
       int issued_k = 0, issued_v = 0;
-      for (int it = 0; it < U; ++it) {
-        const int j = ubhi - 1 - it;
-        const int slot = it % L::STAGES;
-        const uint32_t ph = uint32_t(it / L::STAGES) & 1u;
-        if (!mbar_wait(bar(L::B_KE + slot), ph ^ 1u, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(L::B_KF + slot), L::TILE);
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_4d(sb + L::OFF_K + slot * L::TILE + c * L::HALF, &tmK, bar(L::B_KF + slot),
-                      c * 64, hkv, j * 128, b);
-        issued_k = it + 1;
-        if (!mbar_wait(bar(L::B_VE + slot), ph ^ 1u, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(L::B_VF + slot), L::TILE);
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_4d(sb + L::OFF_V + slot * L::TILE + c * L::HALF, &tmV, bar(L::B_VF + slot),
-                      c * 64, hkv, j * 128, b);
-        issued_v = it + 1;
+      bool alive = true;
+      for (int k = 0; alive; ++k) {
+        const int item = item_of(p, k);
+        if (item < 0) break;
+        WorkItem w;
+        decode_item(p, item, w);
+        if (w.U == 0) continue;
+        // Q buffers are free once every Q.K^T of the previous item completed
+        if (qi > 0 && !(alive = mbar_wait(bar(L::B_QE), uint32_t((qi - 1) & 1), abort_flag))) break;
+        mbar_arrive_expect_tx(bar(L::B_Q), 2 * L::TILE);
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_4d(sb + L::OFF_Q + t * L::TILE + c * L::HALF, &tmQ, bar(L::B_Q), c * 64,
+                        w.tile[t].hq, w.tile[t].row0, w.b);
+        ++qi;
+        for (int it = 0; it < w.U; ++it, ++kv) {
+          const int j = w.ubhi - 1 - it;
+          const int slot = kv % L::STAGES;
+          const uint32_t ph = uint32_t(kv / L::STAGES) & 1u;
+          if (!(alive = mbar_wait(bar(L::B_KE + slot), ph ^ 1u, abort_flag))) break;
+          mbar_arrive_expect_tx(bar(L::B_KF + slot), L::TILE);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_4d(sb + L::OFF_K + slot * L::TILE + c * L::HALF, &tmK, bar(L::B_KF + slot),
+                        c * 64, w.hkv, j * 128, w.b);
+          issued_k = kv + 1;
+          if (!(alive = mbar_wait(bar(L::B_VE + slot), ph ^ 1u, abort_flag))) break;
+          mbar_arrive_expect_tx(bar(L::B_VF + slot), L::TILE);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_4d(sb + L::OFF_V + slot * L::TILE + c * L::HALF, &tmV, bar(L::B_VF + slot),
+                        c * 64, w.hkv, j * 128, w.b);
+          issued_v = kv + 1;
+        }
       }
       // Make sure no copy is still landing in shared memory at exit: wait for
       // the most recent phase of every stage (already complete normally).
-      mbar_wait(bar(L::B_Q), 0, nullptr);
+      if (qi > 0) mbar_wait(bar(L::B_Q), uint32_t((qi - 1) & 1), nullptr);
       for (int it = max(0, issued_k - L::STAGES); it < issued_k; ++it)
         mbar_wait(bar(L::B_KF + it % L::STAGES), uint32_t(it / L::STAGES) & 1u, nullptr);
       for (int it = max(0, issued_v - L::STAGES); it < issued_v; ++it)
