@@ -205,13 +205,19 @@ int decode_group_tile(int G) {
 }
 
 // Split count chosen from sizes alone (so the workspace size needs no Hkv):
-// enough CTAs for several waves over the SMs, each streaming >= 256 keys.
+// assuming work items of four query heads, the smallest split count whose
+// items spread over the SMs with at least 95% balance (persistent CTAs take
+// items round-robin), each item streaming at least one 128-key tile.
 int auto_splits(int B, int Hq, int Lmax) {
-  const long long items = std::max(1ll, (static_cast<long long>(B) * Hq + 3) / 4);
-  long long s = (static_cast<long long>(kNumSMs) * 8 + items - 1) / items;
-  const long long cap = std::max(1, (Lmax + 255) / 256);
-  s = std::min(std::max(s, 1ll), cap);
-  return static_cast<int>(std::min(s, 256ll));
+  const long long base = std::max(1ll, (static_cast<long long>(B) * Hq + 3) / 4);
+  const int cap = std::max(1, std::min(64, (Lmax + 127) / 128));
+  int best = cap;
+  for (int s = 1; s <= cap; ++s) {
+    const long long items = base * s;
+    const long long rounds = (items + kNumSMs - 1) / kNumSMs;
+    if (items >= kNumSMs && double(items) / double(rounds * kNumSMs) >= 0.95) { best = s; break; }
+  }
+  return best;
 }
 
 struct DecodeShape {
@@ -224,7 +230,7 @@ DecodeShape decode_shape(int B, int Hq, int d, int num_splits, int Lmax) {
   DecodeShape s{};
   int S = num_splits > 0 ? num_splits : auto_splits(B, Hq, Lmax);
   if (S > Lmax) S = Lmax;
-  const int quantum = (d == 128) ? 32 : 64;         // keys per CTA block of passes
+  const int quantum = 128;                          // keys per K/V tile
   int chunk = (Lmax + S - 1) / S;
   chunk = (chunk + quantum - 1) / quantum * quantum;
   S = (Lmax + chunk - 1) / chunk;
@@ -238,12 +244,32 @@ DecodeShape decode_shape(int B, int Hq, int d, int num_splits, int Lmax) {
 }
 
 template <int D, int GT>
-void launch_decode_kernels(const attn::DecodeParams& p, cudaStream_t stream) {
+int launch_decode_kernels(attn::DecodeParams& p, const void* k_cache, const void* v_cache,
+                          cudaStream_t stream, int dev) {
+  using L = attn::DecLayout<D>;
+  CUtensorMap mk, mv;
+  int rc;
+  if ((rc = make_map(&mk, k_cache, D, p.Hkv, p.Lmax, p.B)) != ATTN_OK) return rc;
+  if ((rc = make_map(&mv, v_cache, D, p.Hkv, p.Lmax, p.B)) != ATTN_OK) return rc;
   const int G = p.Hq / p.Hkv;
-  dim3 grid_split(p.S, p.Hkv * (G / GT), p.B);
-  attn::decode_split_kernel<D, GT><<<grid_split, attn::kDecodeThreads, 0, stream>>>(p);
+  const long long items = static_cast<long long>(p.B) * p.Hkv * (G / GT) * p.S;
+  if (items > kMaxIndex) return fail(ATTN_ERR_INVALID_ARG, "decode problem too large");
+  p.n_items = static_cast<int>(items);
+  int sms = 0;
+  if ((rc = sm_count(dev, &sms)) != ATTN_OK) return rc;
+  static std::atomic<unsigned long long> attr_set{0};   // per-device bit
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(attr_set.load() & bit)) {
+    cudaError_t e = cudaFuncSetAttribute(attn::decode_split_kernel<D, GT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_ALLOC);
+    if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    attr_set.fetch_or(bit);
+  }
+  const int grid = static_cast<int>(std::min<long long>(items, sms));
+  attn::decode_split_kernel<D, GT><<<grid, attn::kDecodeSplitThreads, L::SMEM_ALLOC, stream>>>(mk, mv, p);
   const int n = p.B * p.Hq;
   attn::decode_combine_kernel<D><<<(n + 3) / 4, 128, 0, stream>>>(p);
+  return ATTN_OK;
 }
 
 // ------------------------------------------------------ no-alloc decode --
@@ -320,14 +346,15 @@ int attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
   p.scale_log2 = scale * 1.4426950408889634f;
   const int GT = decode_group_tile(Hq / Hkv);
   if (d == 128) {
-    if (GT == 4) launch_decode_kernels<128, 4>(p, stream);
-    else if (GT == 2) launch_decode_kernels<128, 2>(p, stream);
-    else launch_decode_kernels<128, 1>(p, stream);
+    if (GT == 4) rc = launch_decode_kernels<128, 4>(p, k_cache, v_cache, stream, dev);
+    else if (GT == 2) rc = launch_decode_kernels<128, 2>(p, k_cache, v_cache, stream, dev);
+    else rc = launch_decode_kernels<128, 1>(p, k_cache, v_cache, stream, dev);
   } else {
-    if (GT == 4) launch_decode_kernels<64, 4>(p, stream);
-    else if (GT == 2) launch_decode_kernels<64, 2>(p, stream);
-    else launch_decode_kernels<64, 1>(p, stream);
+    if (GT == 4) rc = launch_decode_kernels<64, 4>(p, k_cache, v_cache, stream, dev);
+    else if (GT == 2) rc = launch_decode_kernels<64, 2>(p, k_cache, v_cache, stream, dev);
+    else rc = launch_decode_kernels<64, 1>(p, k_cache, v_cache, stream, dev);
   }
+  if (rc != ATTN_OK) return rc;
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "attn_decode_noalloc launch: %s", cudaGetErrorString(e));
   g_launches.fetch_add(2);
@@ -395,14 +422,15 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache, void* o
   p.scale_log2 = scale * 1.4426950408889634f;
   const int GT = decode_group_tile(Hq / Hkv);
   if (d == 128) {
-    if (GT == 4) launch_decode_kernels<128, 4>(p, stream);
-    else if (GT == 2) launch_decode_kernels<128, 2>(p, stream);
-    else launch_decode_kernels<128, 1>(p, stream);
+    if (GT == 4) rc = launch_decode_kernels<128, 4>(p, k_cache, v_cache, stream, dev);
+    else if (GT == 2) rc = launch_decode_kernels<128, 2>(p, k_cache, v_cache, stream, dev);
+    else rc = launch_decode_kernels<128, 1>(p, k_cache, v_cache, stream, dev);
   } else {
-    if (GT == 4) launch_decode_kernels<64, 4>(p, stream);
-    else if (GT == 2) launch_decode_kernels<64, 2>(p, stream);
-    else launch_decode_kernels<64, 1>(p, stream);
+    if (GT == 4) rc = launch_decode_kernels<64, 4>(p, k_cache, v_cache, stream, dev);
+    else if (GT == 2) rc = launch_decode_kernels<64, 2>(p, k_cache, v_cache, stream, dev);
+    else rc = launch_decode_kernels<64, 1>(p, k_cache, v_cache, stream, dev);
   }
+  if (rc != ATTN_OK) return rc;
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "attn_decode launch: %s", cudaGetErrorString(e));
   g_launches.fetch_add(2);
