@@ -59,8 +59,8 @@ struct FwdLayout {
   static constexpr int B_VF = B_KE + STAGES;
   static constexpr int B_VE = B_VF + STAGES;
   static constexpr int B_SF = B_VE + STAGES;            // + tile
-  static constexpr int B_PF = B_SF + 2;
-  static constexpr int B_OD = B_PF + 2;                 // P.V done, + tile
+  static constexpr int B_PF = B_SF + 2;                 // P written, + 2 * tile + key half
+  static constexpr int B_OD = B_PF + 4;                 // P.V done, + tile
   static constexpr int B_OE = B_OD + 2;                 // O read by the epilogue, + tile
   static constexpr int B_DRAIN = B_OE + 2;
   static constexpr int NBAR = B_DRAIN + 1;
@@ -139,12 +139,14 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_smem, uint3
   }
 }
 
+// O += P V for keys [64 hf, 64 hf + 64) of the tile (four MMAs of 16 keys).
 template <int D>
-__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_smem,
-                                         bool accumulate) {
+__device__ __forceinline__ void issue_pv_half(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_smem,
+                                              int hf, bool accumulate) {
   using L = FwdLayout<D>;
 #pragma unroll
-  for (int k = 0; k < 128 / 16; ++k) {
+  for (int kk = 0; kk < 4; ++kk) {
+    const int k = 4 * hf + kk;
     const uint64_t b = smem_desc_sw128(v_smem + k * 16 * 128, L::HALF, 1024);
     mma_ts(d_tmem, p_tmem + 8 * k, b, L::IDESC_PV, (accumulate || k > 0) ? 1u : 0u);
   }
@@ -234,7 +236,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar(L::B_SF + t), 1);
-      mbar_init(bar(L::B_PF + t), 128);
+      mbar_init(bar(L::B_PF + 2 * t + 0), 128);
+      mbar_init(bar(L::B_PF + 2 * t + 1), 128);
       mbar_init(bar(L::B_OD + t), 1);
       mbar_init(bar(L::B_OE + t), 128);
     }
@@ -304,19 +307,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           for (int c = 0; c < 128; ++c)
             if (c < lo_rel || c > hi_rel) s[c] = -CUDART_INF_F;
         }
-        // row max: 8 independent chains of 3-input max
+        // row max: 8 independent chains
         float mx[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) mx[i] = s[i];
 #pragma unroll
-        for (int c = 8; c < 120; c += 16) {
+        for (int c = 8; c < 128; c += 8) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) mx[i] = max3f(mx[i], s[c + i], s[c + 8 + i]);
+          for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[c + i]);
         }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[120 + i]);
-        const float mb = fmaxf(max3f(mx[0], mx[1], mx[2]),
-                               fmaxf(max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        const float mb = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
         // Lazy rescale: keep the old maximum while the new one exceeds it by at
         // most 8 in log2 units (P values stay <= 256); the final O / l is exact
         // whichever maximum was used.
@@ -329,53 +330,59 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         }
         const float mo = (m == -CUDART_INF_F) ? 0.f : m * c2;
         // P = 2^(s * c2 - mo) on pairs; in unmasked tiles every kPolyEvery-th
-        // pair goes to the FMA-pipe polynomial to offload the MUFU unit.
+        // pair goes to the FMA-pipe polynomial to offload the MUFU unit. P is
+        // written and announced in two halves of 64 keys so the tensor core
+        // starts P.V on the first half while the second is computed.
         const uint64_t C2 = f2_pack(c2, c2), NMO = f2_pack(-mo, -mo);
         uint64_t lacc[4] = {0, 0, 0, 0};
-        uint32_t pk[64];
-        if (masked) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            const float2 x = f2_unpack(f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), C2, NMO));
-            const float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
-            lacc[c & 3] = f2_add(lacc[c & 3], f2_pack(p0, p1));
-            pk[c] = pack_bf16x2(p0, p1);
-          }
-        } else {
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t pk[32];
+          if (masked) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            const uint64_t x = f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), C2, NMO);
-            uint64_t e;
-            if ((c % kPolyEvery) == kPolyEvery - 1) {
-              e = exp2_poly_f2(x);
-            } else {
-              const float2 xx = f2_unpack(x);
-              e = f2_pack(ex2_approx(xx.x), ex2_approx(xx.y));
+            for (int i = 0; i < 32; ++i) {
+              const int c = 32 * hf + i;
+              const float2 x = f2_unpack(f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), C2, NMO));
+              const float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
+              lacc[i & 3] = f2_add(lacc[i & 3], f2_pack(p0, p1));
+              pk[i] = pack_bf16x2(p0, p1);
             }
-            lacc[c & 3] = f2_add(lacc[c & 3], e);
-            const float2 ee = f2_unpack(e);
-            pk[c] = pack_bf16x2(ee.x, ee.y);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int c = 32 * hf + i;
+              const uint64_t x = f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), C2, NMO);
+              uint64_t e;
+              if ((i % kPolyEvery) == kPolyEvery - 1) {
+                e = exp2_poly_f2(x);
+              } else {
+                const float2 xx = f2_unpack(x);
+                e = f2_pack(ex2_approx(xx.x), ex2_approx(xx.y));
+              }
+              lacc[i & 3] = f2_add(lacc[i & 3], e);
+              const float2 ee = f2_unpack(e);
+              pk[i] = pack_bf16x2(ee.x, ee.y);
+            }
           }
+          tmem_st32(tS + 32 * hf, pk);
+          if (hf == 0 && n_in_item > 0 && __any_sync(0xffffffffu, rescale)) {
+            // O must be rescaled before the first half's P.V accumulates
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t o[32];
+              tmem_ld32(tO + 32 * c, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              tmem_st32(tO + 32 * c, o);
+            }
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(bar(L::B_PF + 2 * t + hf));
         }
         const float2 l01 = f2_unpack(f2_add(f2_add(lacc[0], lacc[1]), f2_add(lacc[2], lacc[3])));
         l = fmaf(l, alpha, l01.x + l01.y);
-        tmem_st32(tS, pk);
-        tmem_st32(tS + 32, pk + 32);
-
-        if (n_in_item > 0 && __any_sync(0xffffffffu, rescale)) {
-#pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tO + 32 * c, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(tO + 32 * c, o);
-          }
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(bar(L::B_PF + t));
         ++count;
         ++n_in_item;
       }
@@ -432,8 +439,26 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const uint32_t q0 = sb + L::OFF_Q, q1 = sb + L::OFF_Q + L::TILE;
       const uint32_t dS0 = tmem + L::COL_S0, dS1 = tmem + L::COL_S1;
       const uint32_t dO0 = tmem + L::COL_O0, dO1 = tmem + L::COL_O1;
-      int pv0 = 0, pv1 = 0;                 // P.V products issued per tile (all items)
-      int done0 = 0, done1 = 0;             // items in which each tile had work
+      int pv[2] = {0, 0};                   // P.V products issued per tile (all items)
+      int done[2] = {0, 0};                 // items in which each tile had work
+      bool first[2] = {true, true};         // no P.V of the tile yet in this item
+      // O_t += P_t V: each 64-key half as soon as the softmax has written it
+      auto pv_tile = [&](int t, int vslot) -> bool {
+        const uint32_t vsm = sb + L::OFF_V + vslot * L::TILE;
+        const uint32_t dO = t ? dO1 : dO0, dS = t ? dS1 : dS0;
+        if (!mbar_wait(bar(L::B_PF + 2 * t + 0), uint32_t(pv[t] & 1), abort_flag)) return false;
+        if (first[t] && done[t] > 0 &&
+            !mbar_wait(bar(L::B_OE + t), uint32_t((done[t] - 1) & 1), abort_flag)) return false;
+        tc_fence_after();
+        issue_pv_half<D>(dO, dS, vsm, 0, !first[t]);
+        if (!mbar_wait(bar(L::B_PF + 2 * t + 1), uint32_t(pv[t] & 1), abort_flag)) return false;
+        tc_fence_after();
+        issue_pv_half<D>(dO, dS, vsm, 1, true);
+        tc_commit(bar(L::B_OD + t));
+        ++pv[t];
+        first[t] = false;
+        return true;
+      };
       int kv = 0, qi = 0;                   // K/V ring position, items with a Q load
       bool alive = true;
       for (int k = 0; alive; ++k) {
@@ -444,7 +469,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (w.U == 0) continue;
         if (!(alive = mbar_wait(bar(L::B_Q), uint32_t(qi & 1), abort_flag))) break;
         tc_fence_after();
-        bool first0 = true, first1 = true;
+        first[0] = first[1] = true;
         int prev_j = -1, prev_slot = 0;
         for (int it = 0; it < w.U; ++it, ++kv) {
           const int j = w.ubhi - 1 - it;
@@ -458,16 +483,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             tc_commit(bar(L::B_SF + 0));
           }
           if (it > 0) {
-            if (tile_has(w.tile[1], prev_j)) {
-              if (!(alive = mbar_wait(bar(L::B_PF + 1), uint32_t(pv1 & 1), abort_flag))) break;
-              if (first1 && done1 > 0 &&
-                  !(alive = mbar_wait(bar(L::B_OE + 1), uint32_t((done1 - 1) & 1), abort_flag))) break;
-              tc_fence_after();
-              issue_pv<D>(dO1, dS1, sb + L::OFF_V + prev_slot * L::TILE, !first1);
-              tc_commit(bar(L::B_OD + 1));
-              ++pv1;
-              first1 = false;
-            }
+            if (tile_has(w.tile[1], prev_j) && !(alive = pv_tile(1, prev_slot))) break;
             tc_commit(bar(L::B_VE + prev_slot));
           }
           if (tile_has(w.tile[1], j)) {
@@ -478,33 +494,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           if (it == w.U - 1) tc_commit(bar(L::B_QE));     // every Q.K^T of this item issued
           if (!(alive = mbar_wait(bar(L::B_VF + slot), ph, abort_flag))) break;
           tc_fence_after();
-          if (tile_has(w.tile[0], j)) {
-            if (!(alive = mbar_wait(bar(L::B_PF + 0), uint32_t(pv0 & 1), abort_flag))) break;
-            if (first0 && done0 > 0 &&
-                !(alive = mbar_wait(bar(L::B_OE + 0), uint32_t((done0 - 1) & 1), abort_flag))) break;
-            tc_fence_after();
-            issue_pv<D>(dO0, dS0, sb + L::OFF_V + slot * L::TILE, !first0);
-            tc_commit(bar(L::B_OD + 0));
-            ++pv0;
-            first0 = false;
-          }
+          if (tile_has(w.tile[0], j) && !(alive = pv_tile(0, slot))) break;
           prev_j = j;
           prev_slot = slot;
         }
         if (!alive) break;
-        if (tile_has(w.tile[1], prev_j)) {
-          if (!(alive = mbar_wait(bar(L::B_PF + 1), uint32_t(pv1 & 1), abort_flag))) break;
-          if (first1 && done1 > 0 &&
-              !(alive = mbar_wait(bar(L::B_OE + 1), uint32_t((done1 - 1) & 1), abort_flag))) break;
-          tc_fence_after();
-          issue_pv<D>(dO1, dS1, sb + L::OFF_V + prev_slot * L::TILE, !first1);
-          tc_commit(bar(L::B_OD + 1));
-          ++pv1;
-          first1 = false;
-        }
+        if (tile_has(w.tile[1], prev_j) && !(alive = pv_tile(1, prev_slot))) break;
         tc_commit(bar(L::B_VE + prev_slot));
-        if (!first0) ++done0;
-        if (!first1) ++done1;
+        if (!first[0]) ++done[0];
+        if (!first[1]) ++done[1];
         ++qi;
       }
       // drain: every issued tensor-core operation completes before teardown
