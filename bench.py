@@ -182,11 +182,23 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The slowest rank's value (timings are reported as the max over ranks)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def shard_seed(rank: int) -> int:
+    """Each rank draws its own batch: independent shards, no data exchanged."""
+    return ai.SEED_Q + 17 * rank
+
+
+def whole_job_rate(units_per_rank: float, ms_max: float, world: int) -> float:
+    """Units per second of the whole job: all ranks' units over the slowest rank's time."""
+    return world * units_per_rank / (ms_max * 1e-3)
 
 
 # ------------------------------------------------------------------ timing --
@@ -339,7 +351,7 @@ def run_ours(args, world, rank, local):
     w = PREFILL[args.workload]
     if args.batch:
         w = dataclasses.replace(w, B=args.batch, name=f"{w.name} [batch {args.batch}]")
-    q_h, k_h, v_h = ai.make_for(w, seed=ai.SEED_Q + 17 * rank)
+    q_h, k_h, v_h = ai.make_for(w, seed=shard_seed(rank))
     q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
     o = torch.empty((w.B, w.Nq, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=dev)
@@ -355,7 +367,7 @@ def run_ours(args, world, rank, local):
     ms = statistics.mean(times)
     ms_max = max_over_ranks(ms, world)
     flops = metrics.attn_flops(w.B, w.Hq, w.Nq, w.Nk, w.d, w.causal, w.window_left)
-    value = world * flops / (ms_max * 1e-3) / 1e12
+    value = whole_job_rate(flops, ms_max, world) / 1e12
     achieved = flops / (ms * 1e-3) / 1e12
     tiles = metrics.executed_tiles(w.Nq, w.Nk, w.causal, w.window_left) * w.B * w.Hq
     clocks = sampler.summary()
@@ -364,7 +376,7 @@ def run_ours(args, world, rank, local):
     dw = ai.GQA_DECODE
     if args.decode_batch:
         dw = dataclasses.replace(dw, B=args.decode_batch, name=f"{dw.name} [batch {args.decode_batch}]")
-    qd_h, kc_h, vc_h = ai.make_decode(dw.B, dw.Hq, dw.Hkv, dw.Nk, dw.d, seed=ai.SEED_Q + 17 * rank)
+    qd_h, kc_h, vc_h = ai.make_decode(dw.B, dw.Hq, dw.Hkv, dw.Nk, dw.d, seed=shard_seed(rank))
     qd, kc, vc = qd_h.to(dev), kc_h.to(dev), vc_h.to(dev)
     od = torch.empty((dw.B, dw.Hq, dw.d), dtype=torch.bfloat16, device=dev)
     lsed = torch.empty((dw.B, dw.Hq), dtype=torch.float32, device=dev)
@@ -380,7 +392,7 @@ def run_ours(args, world, rank, local):
     dms_max = max_over_ranks(dms, world)
     kv_bytes = metrics.decode_kv_bytes([dw.Nk] * dw.B, dw.Hkv, dw.d)
     d_all = metrics.decode_bytes(dw.B, dw.Hq, dw.Hkv, [dw.Nk] * dw.B, dw.d)
-    d_value = world * kv_bytes / (dms_max * 1e-3) / 1e9
+    d_value = whole_job_rate(kv_bytes, dms_max, world) / 1e9
 
     # end-to-end through the public API with host buffers
     e2e = None
@@ -400,7 +412,7 @@ def run_ours(args, world, rank, local):
         e_ms = max_over_ranks(e2e_loop(e2e_step, min(args.steps, 30), 2), world)
         h2d = sum(t.numel() * t.element_size() for t in (qp, kp, vp))
         d2h = op.numel() * op.element_size() + lp.numel() * lp.element_size()
-        e2e = {"value": world * flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": whole_job_rate(flops, e_ms, world) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
 
     cpu = None

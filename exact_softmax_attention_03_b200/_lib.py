@@ -42,6 +42,7 @@ SIGNATURES = {
                                  _vp]),
     "attn_last_error": (ctypes.c_char_p, []),
     "attn_device_status": (_i, [_vp]),
+    "attn_selftest_wait_timeout": (_i, [_vp]),
     "attn_launch_count": (ctypes.c_ulonglong, []),
 }
 

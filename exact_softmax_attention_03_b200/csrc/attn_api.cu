@@ -450,6 +450,17 @@ int attn_device_status(cudaStream_t stream) {
   return ok();
 }
 
+int attn_selftest_wait_timeout(cudaStream_t stream) {
+  int dev = 0;
+  int rc = check_device(&dev);
+  if (rc != ATTN_OK) return rc;
+  attn::selftest_wait_kernel<<<1, 32, 0, stream>>>();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "selftest launch: %s", cudaGetErrorString(e));
+  g_launches.fetch_add(1);
+  return ok();
+}
+
 unsigned long long attn_launch_count(void) { return g_launches.load(); }
 
 }  // extern "C"

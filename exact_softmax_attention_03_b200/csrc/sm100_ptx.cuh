@@ -83,6 +83,22 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   return mbar_wait_slow(bar, parity, abort);
 }
 
+// Waits on a barrier that nothing completes: the bounded wait gives up after
+// kWaitLimitNs and records ATTN_ERR_TIMEOUT in the status word (used to test
+// the failure-detection path without faulting or hanging the GPU).
+__global__ void selftest_wait_kernel() {
+  __shared__ uint64_t never;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&never), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(smem_u32(&never), 0, &abort_flag);
+  __syncthreads();
+}
+
 // Named barrier over `count` threads (a warpgroup uses 128).
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");

@@ -150,6 +150,17 @@ const char* attn_last_error(void);
  */
 int attn_device_status(cudaStream_t stream);
 
+/*
+ * Diagnostic for the failure-detection path. Launches one small kernel whose
+ * thread waits on a shared-memory barrier that nothing ever completes. The
+ * wait is bounded like every wait in this library's kernels: after about one
+ * second it gives up, sets the device status word and the kernel returns, so
+ * the context stays usable. A following attn_device_status(stream) then
+ * returns ATTN_ERR_TIMEOUT (and clears the word). Returns ATTN_OK when the
+ * launch was issued.
+ */
+int attn_selftest_wait_timeout(cudaStream_t stream);
+
 /* Number of kernel launches this library has issued in this process. */
 unsigned long long attn_launch_count(void);
 

@@ -33,7 +33,8 @@ def header_functions():
 def test_header_declares_the_expected_entry_points():
     assert header_functions() == sorted([
         "attn_fwd", "attn_fwd_f32o", "attn_decode_workspace_bytes", "attn_decode",
-        "attn_decode_noalloc", "attn_last_error", "attn_device_status", "attn_launch_count"])
+        "attn_decode_noalloc", "attn_last_error", "attn_device_status", "attn_launch_count",
+        "attn_selftest_wait_timeout"])
 
 
 def test_library_exports_every_declared_symbol(lib):

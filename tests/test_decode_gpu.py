@@ -50,7 +50,7 @@ def test_decode_split_counts(num_splits):
 
 
 @pytest.mark.parametrize("Hq,Hkv,d", [(8, 8, 128), (8, 1, 128), (6, 2, 128), (8, 4, 64),
-                                      (16, 2, 64), (3, 3, 64)])
+                                      (16, 2, 64), (3, 3, 64), (32, 4, 128), (32, 1, 128)])
 def test_decode_head_layouts(Hq, Hkv, d):
     check(3, Hq, Hkv, 777, d)
 

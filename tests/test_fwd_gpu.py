@@ -70,6 +70,9 @@ SHAPES = [
     ((1, 1, 1, 2048, 2048, 128), False, -1),
     ((1, 2, 2, 700, 1500, 128), False, 300),
     ((1, 2, 2, 1, 4000, 128), True, -1),         # one query at the end of a long key set
+    ((1, 16, 2, 257, 257, 128), True, 100),      # GQA group of 8: four head pairs per K/V head
+    ((2, 32, 1, 200, 200, 64), False, -1),       # MQA, 32 query heads on one K/V head
+    ((3, 4, 2, 129, 385, 64), True, 64),         # ragged, Nq < Nk, window, d = 64
 ]
 
 
