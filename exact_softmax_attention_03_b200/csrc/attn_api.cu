@@ -167,8 +167,15 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   static std::atomic<unsigned long long> attr_set{0};   // per-device bit
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(attr_set.load() & bit)) {
-    cudaError_t e = cudaFuncSetAttribute(attn::attn_fwd_kernel<D, F32OUT>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_ALLOC);
+    // the in-kernel register split needs this many registers per thread at launch
+    cudaFuncAttributes fa{};
+    cudaError_t e = cudaFuncGetAttributes(&fa, attn::attn_fwd_kernel<D, F32OUT>);
+    if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "cudaFuncGetAttributes: %s", cudaGetErrorString(e));
+    if (fa.numRegs < attn::kFwdRegsLaunchMin)
+      return fail(ATTN_ERR_UNSUPPORTED, "attn_fwd kernel built with %d registers per thread, needs %d",
+                  fa.numRegs, attn::kFwdRegsLaunchMin);
+    e = cudaFuncSetAttribute(attn::attn_fwd_kernel<D, F32OUT>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_ALLOC);
     if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     attr_set.fetch_or(bit);
   }

@@ -88,6 +88,24 @@ struct FwdParams {
 };
 
 constexpr int kFwdThreads = 384;
+// Register split: the two softmax warpgroups hold a 128-score row each and
+// take kFwdRegsSoftmax per thread; the issuer/producer warpgroup gives its
+// registers up down to kFwdRegsOther (192 / 112 is the split at which neither
+// side spills). The launch must have at least kFwdRegsLaunchMin registers per
+// thread for the split to fit; the host checks the built kernel's count.
+#ifndef ATTN_REGS_SM
+#define ATTN_REGS_SM 192
+#endif
+#ifndef ATTN_REGS_OT
+#define ATTN_REGS_OT 112
+#endif
+constexpr int kFwdRegsSoftmax = ATTN_REGS_SM;
+constexpr int kFwdRegsOther = ATTN_REGS_OT;
+constexpr int kFwdRegsLaunch = 168;     // 65536 / 384 rounded down to a multiple of 8
+constexpr int kFwdRegsLaunchMin = (2 * 128 * kFwdRegsSoftmax + 128 * kFwdRegsOther + kFwdThreads - 1) / kFwdThreads;
+#ifndef ATTN_PROBE_REGS
+static_assert(kFwdRegsLaunchMin <= kFwdRegsLaunch, "register split exceeds the launch budget");
+#endif
 // Every kPolyEvery-th pair of exponentials in an unmasked score tile is
 // computed on the FMA pipe instead of the MUFU unit.
 #ifndef ATTN_POLY_EVERY
@@ -256,6 +274,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
   if (warp < 8) {
     // ======================= softmax warpgroups ==============================
+    reg_alloc<kFwdRegsSoftmax>();
     const int t = warp >> 2;
     const int row = int(threadIdx.x) - 128 * t;
     const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
@@ -269,7 +288,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       if (item < 0) break;
       WorkItem w;
       decode_item(p, item, w);
-      const TileInfo& T = w.tile[t];
+      const TileInfo T = t ? w.tile[1] : w.tile[0];   // by value: no local-memory copy of w
       if (!T.active) continue;
       const int r = T.row0 + row;
       const int qpos = r + p.Nk - p.Nq;
@@ -277,12 +296,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       float l = 0.f;                        // running sum of exp2((s - m) * c2)
       int n_in_item = 0;
       for (int j = T.bhi - 1; j >= T.blo; --j) {
-        bool wt = mbar_wait(bar(L::B_SF + t), uint32_t(count & 1), abort_flag);
+        bool wt = mbar_wait<1>(bar(L::B_SF + t), uint32_t(count & 1), abort_flag);
         // the previous P.V of this item must be done before P is overwritten
         // and before O is rescaled (at an item's first tile it was waited for
         // in the previous epilogue)
         if (wt && n_in_item > 0)
-          wt = mbar_wait(bar(L::B_OD + t), uint32_t((count - 1) & 1), abort_flag);
+          wt = mbar_wait<1>(bar(L::B_OD + t), uint32_t((count - 1) & 1), abort_flag);
         if (!__all_sync(0xffffffffu, wt)) { ok = false; break; }
         tc_fence_after();
 
@@ -391,7 +410,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       // ---- epilogue: O / l and LSE -----------------------------------------
       bool have = n_in_item > 0;
       if (have) {
-        const bool wt = mbar_wait(bar(L::B_OD + t), uint32_t((count - 1) & 1), abort_flag);
+        const bool wt = mbar_wait<1>(bar(L::B_OD + t), uint32_t((count - 1) & 1), abort_flag);
         if (!__all_sync(0xffffffffu, wt)) { ok = false; break; }
         tc_fence_after();
       }
@@ -433,7 +452,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
               (l > 0.f) ? fmaf(m, p.scale, __log2f(l) * 0.6931471805599453f) : -CUDART_INF_F;
       }
     }
-  } else if (warp == 8) {
+  } else {
+  // warps 8-11 release registers to the softmax warpgroups (the release is
+  // larger than the softmax groups' increase)
+  reg_dealloc<kFwdRegsOther>();
+  if (warp == 8) {
     // ======================= tensor-core issuer ==============================
     if (lane == 0) {
       const uint32_t q0 = sb + L::OFF_Q, q1 = sb + L::OFF_Q + L::TILE;
@@ -562,8 +585,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
     __syncwarp();
   }
+  }
 
   // ---- teardown --------------------------------------------------------------
+  // (register budgets stay split: no warpgroup increases its budget again, so
+  // the only increase, the softmax groups' at the start, is always granted)
   tc_fence_before();
   __syncthreads();
   if (warp == 8) {

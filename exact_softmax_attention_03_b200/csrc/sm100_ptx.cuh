@@ -59,6 +59,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Slow path of mbar_wait (kept out of line so the fast path stays cheap).
+// Code running under different per-warpgroup register budgets (setmaxnreg)
+// must call different instances of an out-of-line function: `Region` tells
+// them apart.
+template <int Region>
 __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort) {
   const unsigned long long t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
@@ -78,9 +82,10 @@ __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volat
 // kWaitLimitNs, or as soon as *abort (if not null) is set by another thread of
 // the CTA; on a timeout it sets *abort and the device status word. Returns
 // whether the phase completed.
+template <int Region = 0>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
-  return mbar_wait_slow(bar, parity, abort);
+  return mbar_wait_slow<Region>(bar, parity, abort);
 }
 
 // Waits on a barrier that nothing completes: the bounded wait gives up after
@@ -130,6 +135,18 @@ __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
 }
 __device__ __forceinline__ void tmem_relinquish() {
   asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+// Per-warpgroup register budget (all four warps of a warpgroup execute the
+// same one). An increase is granted from the registers that other warpgroups
+// of the CTA released, so the launch's registers per thread must cover the
+// split; the host checks that before the launch.
+template <uint32_t N>
+__device__ __forceinline__ void reg_alloc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void reg_dealloc() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)

@@ -134,3 +134,35 @@ def test_full_size_sampled_rows(w):
         O, L = oracle.oracle_attention_rows(q, k, v, b, hq, rows, causal=w.causal,
                                             window_left=w.window_left)
         assert_close(o[b, rows, hq], O, lse[b, hq, rows], L, what=(w.name, b, hq))
+
+
+def _scaled_keys(k, factor_of_key):
+    k = k.float().clone()
+    for j in range(k.shape[1]):
+        f = factor_of_key(j)
+        if f != 1.0:
+            k[:, j] *= f
+    return k.to(torch.bfloat16)
+
+
+def test_scores_growing_across_blocks_force_a_fresh_max():
+    # Key blocks are visited from the last one backwards; the early keys get
+    # scores tens of log2 units above everything seen before, so the running
+    # max (reused without a max pass) must be refreshed exactly.
+    q, k, v = ai.make_qkv(1, 2, 2, 640, 640, 128)
+    k = _scaled_keys(k, lambda j: 90.0 if j < 128 else (30.0 if j < 256 else 1.0))
+    for causal in (True, False):
+        o, lse = run_fwd(q, k, v, causal, -1)
+        O, L = oracle.oracle_attention(q, k, v, causal=causal)
+        assert_close(o, O, lse, L, what=("growing", causal))
+
+
+def test_overflow_in_second_half_of_a_block():
+    # Only keys 64..127 of block 1 are huge: the first half of that block goes
+    # out with the old max and the second half has to rescale after it.
+    q, k, v = ai.make_qkv(2, 4, 2, 512, 512, 128)
+    k = _scaled_keys(k, lambda j: 60.0 if 192 <= j < 256 else 1.0)
+    for causal, wl in ((True, -1), (False, -1), (True, 300)):
+        o, lse = run_fwd(q, k, v, causal, wl)
+        O, L = oracle.oracle_attention(q, k, v, causal=causal, window_left=wl)
+        assert_close(o, O, lse, L, what=("second half", causal, wl))
