@@ -145,28 +145,30 @@ __device__ __forceinline__ bool block_needs_mask(const FwdParams& p, const TileI
   return kb1 >= p.Nk || (p.causal && kb1 > qf) || (p.window_left >= 0 && kb0 < ql - p.window_left);
 }
 
+// The MMAs take descriptors built once per buffer: a descriptor's start
+// address field is the byte address >> 4, so the descriptor of (address +
+// off) is the buffer's descriptor + off >> 4 (off a multiple of 16 and the
+// sum inside shared memory, which keeps the field below 2^14).
 template <int D>
-__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem) {
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint64_t q_desc, uint64_t k_desc) {
   using L = FwdLayout<D>;
 #pragma unroll
   for (int k = 0; k < D / 16; ++k) {
-    const uint32_t off = (k / 4) * L::HALF + (k % 4) * 32;
-    const uint64_t a = smem_desc_sw128(q_smem + off, 16, 1024);
-    const uint64_t b = smem_desc_sw128(k_smem + off, 16, 1024);
-    mma_ss(d_tmem, a, b, L::IDESC_QK, k > 0 ? 1u : 0u);
+    const uint32_t off = ((k / 4) * L::HALF + (k % 4) * 32) >> 4;
+    mma_ss(d_tmem, q_desc + off, k_desc + off, L::IDESC_QK, k > 0 ? 1u : 0u);
   }
 }
 
 // O += P V for keys [64 hf, 64 hf + 64) of the tile (four MMAs of 16 keys).
 template <int D>
-__device__ __forceinline__ void issue_pv_half(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_smem,
+__device__ __forceinline__ void issue_pv_half(uint32_t d_tmem, uint32_t p_tmem, uint64_t v_desc,
                                               int hf, bool accumulate) {
   using L = FwdLayout<D>;
 #pragma unroll
   for (int kk = 0; kk < 4; ++kk) {
     const int k = 4 * hf + kk;
-    const uint64_t b = smem_desc_sw128(v_smem + k * 16 * 128, L::HALF, 1024);
-    mma_ts(d_tmem, p_tmem + 8 * k, b, L::IDESC_PV, (accumulate || k > 0) ? 1u : 0u);
+    mma_ts(d_tmem, p_tmem + 8 * k, v_desc + ((k * 16 * 128) >> 4), L::IDESC_PV,
+           (accumulate || k > 0) ? 1u : 0u);
   }
 }
 
@@ -459,7 +461,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   if (warp == 8) {
     // ======================= tensor-core issuer ==============================
     if (lane == 0) {
-      const uint32_t q0 = sb + L::OFF_Q, q1 = sb + L::OFF_Q + L::TILE;
+      const uint64_t dq0 = smem_desc_sw128(sb + L::OFF_Q, 16, 1024);
+      const uint64_t dq1 = smem_desc_sw128(sb + L::OFF_Q + L::TILE, 16, 1024);
+      const uint64_t dk = smem_desc_sw128(sb + L::OFF_K, 16, 1024);          // + slot * TILE
+      const uint64_t dv = smem_desc_sw128(sb + L::OFF_V, L::HALF, 1024);     // + slot * TILE
       const uint32_t dS0 = tmem + L::COL_S0, dS1 = tmem + L::COL_S1;
       const uint32_t dO0 = tmem + L::COL_O0, dO1 = tmem + L::COL_O1;
       int pv[2] = {0, 0};                   // P.V products issued per tile (all items)
@@ -467,16 +472,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       bool first[2] = {true, true};         // no P.V of the tile yet in this item
       // O_t += P_t V: each 64-key half as soon as the softmax has written it
       auto pv_tile = [&](int t, int vslot) -> bool {
-        const uint32_t vsm = sb + L::OFF_V + vslot * L::TILE;
+        const uint64_t vd = dv + uint32_t(vslot * (L::TILE >> 4));
         const uint32_t dO = t ? dO1 : dO0, dS = t ? dS1 : dS0;
         if (!mbar_wait(bar(L::B_PF + 2 * t + 0), uint32_t(pv[t] & 1), abort_flag)) return false;
         if (first[t] && done[t] > 0 &&
             !mbar_wait(bar(L::B_OE + t), uint32_t((done[t] - 1) & 1), abort_flag)) return false;
         tc_fence_after();
-        issue_pv_half<D>(dO, dS, vsm, 0, !first[t]);
+        issue_pv_half<D>(dO, dS, vd, 0, !first[t]);
         if (!mbar_wait(bar(L::B_PF + 2 * t + 1), uint32_t(pv[t] & 1), abort_flag)) return false;
         tc_fence_after();
-        issue_pv_half<D>(dO, dS, vsm, 1, true);
+        issue_pv_half<D>(dO, dS, vd, 1, true);
         tc_commit(bar(L::B_OD + t));
         ++pv[t];
         first[t] = false;
@@ -500,9 +505,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           const uint32_t ph = uint32_t(kv / L::STAGES) & 1u;
           if (!(alive = mbar_wait(bar(L::B_KF + slot), ph, abort_flag))) break;
           tc_fence_after();
-          const uint32_t ks = sb + L::OFF_K + slot * L::TILE;
+          const uint64_t kd = dk + uint32_t(slot * (L::TILE >> 4));
           if (tile_has(w.tile[0], j)) {
-            issue_qk<D>(dS0, q0, ks);
+            issue_qk<D>(dS0, dq0, kd);
             tc_commit(bar(L::B_SF + 0));
           }
           if (it > 0) {
@@ -510,7 +515,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             tc_commit(bar(L::B_VE + prev_slot));
           }
           if (tile_has(w.tile[1], j)) {
-            issue_qk<D>(dS1, q1, ks);
+            issue_qk<D>(dS1, dq1, kd);
             tc_commit(bar(L::B_SF + 1));
           }
           tc_commit(bar(L::B_KE + slot));
