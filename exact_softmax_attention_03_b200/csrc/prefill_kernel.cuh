@@ -145,7 +145,8 @@ __device__ __forceinline__ bool block_needs_mask(const FwdParams& p, const TileI
   return kb1 >= p.Nk || (p.causal && kb1 > qf) || (p.window_left >= 0 && kb0 < ql - p.window_left);
 }
 
-// The MMAs take descriptors built once per buffer: a descriptor's start
+// Both are called by the whole issuer warp (warp-uniform operands); one
+// elected lane issues each MMA. The MMAs take descriptors built once per buffer: a descriptor's start
 // address field is the byte address >> 4, so the descriptor of (address +
 // off) is the buffer's descriptor + off >> 4 (off a multiple of 16 and the
 // sum inside shared memory, which keeps the field below 2^14).
@@ -155,7 +156,7 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint64_t q_desc, uint6
 #pragma unroll
   for (int k = 0; k < D / 16; ++k) {
     const uint32_t off = ((k / 4) * L::HALF + (k % 4) * 32) >> 4;
-    mma_ss(d_tmem, q_desc + off, k_desc + off, L::IDESC_QK, k > 0 ? 1u : 0u);
+    if (elect_one()) mma_ss(d_tmem, q_desc + off, k_desc + off, L::IDESC_QK, k > 0 ? 1u : 0u);
   }
 }
 
@@ -167,8 +168,9 @@ __device__ __forceinline__ void issue_pv_half(uint32_t d_tmem, uint32_t p_tmem, 
 #pragma unroll
   for (int kk = 0; kk < 4; ++kk) {
     const int k = 4 * hf + kk;
-    mma_ts(d_tmem, p_tmem + 8 * k, v_desc + ((k * 16 * 128) >> 4), L::IDESC_PV,
-           (accumulate || k > 0) ? 1u : 0u);
+    if (elect_one())
+      mma_ts(d_tmem, p_tmem + 8 * k, v_desc + ((k * 16 * 128) >> 4), L::IDESC_PV,
+             (accumulate || k > 0) ? 1u : 0u);
   }
 }
 
@@ -460,7 +462,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   reg_dealloc<kFwdRegsOther>();
   if (warp == 8) {
     // ======================= tensor-core issuer ==============================
-    if (lane == 0) {
+    // The whole warp runs the loop, so every operand is warp-uniform; one
+    // elected lane (always lane 0) issues each MMA and commit.
+    {
+      // a wait the whole warp agrees on (lanes give up together)
+      auto wwait = [&](int b, uint32_t parity) -> bool {
+        return __all_sync(0xffffffffu, mbar_wait(bar(b), parity, abort_flag));
+      };
+      auto commit = [&](int b) { if (elect_one()) tc_commit(bar(b)); };
       const uint64_t dq0 = smem_desc_sw128(sb + L::OFF_Q, 16, 1024);
       const uint64_t dq1 = smem_desc_sw128(sb + L::OFF_Q + L::TILE, 16, 1024);
       const uint64_t dk = smem_desc_sw128(sb + L::OFF_K, 16, 1024);          // + slot * TILE
@@ -474,15 +483,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       auto pv_tile = [&](int t, int vslot) -> bool {
         const uint64_t vd = dv + uint32_t(vslot * (L::TILE >> 4));
         const uint32_t dO = t ? dO1 : dO0, dS = t ? dS1 : dS0;
-        if (!mbar_wait(bar(L::B_PF + 2 * t + 0), uint32_t(pv[t] & 1), abort_flag)) return false;
+        if (!wwait(L::B_PF + 2 * t + 0, uint32_t(pv[t] & 1))) return false;
         if (first[t] && done[t] > 0 &&
-            !mbar_wait(bar(L::B_OE + t), uint32_t((done[t] - 1) & 1), abort_flag)) return false;
+            !wwait(L::B_OE + t, uint32_t((done[t] - 1) & 1))) return false;
         tc_fence_after();
         issue_pv_half<D>(dO, dS, vd, 0, !first[t]);
-        if (!mbar_wait(bar(L::B_PF + 2 * t + 1), uint32_t(pv[t] & 1), abort_flag)) return false;
+        if (!wwait(L::B_PF + 2 * t + 1, uint32_t(pv[t] & 1))) return false;
         tc_fence_after();
         issue_pv_half<D>(dO, dS, vd, 1, true);
-        tc_commit(bar(L::B_OD + t));
+        commit(L::B_OD + t);
         ++pv[t];
         first[t] = false;
         return true;
@@ -495,7 +504,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         WorkItem w;
         decode_item(p, item, w);
         if (w.U == 0) continue;
-        if (!(alive = mbar_wait(bar(L::B_Q), uint32_t(qi & 1), abort_flag))) break;
+        if (!(alive = wwait(L::B_Q, uint32_t(qi & 1)))) break;
         tc_fence_after();
         first[0] = first[1] = true;
         int prev_j = -1, prev_slot = 0;
@@ -503,24 +512,24 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           const int j = w.ubhi - 1 - it;
           const int slot = kv % L::STAGES;
           const uint32_t ph = uint32_t(kv / L::STAGES) & 1u;
-          if (!(alive = mbar_wait(bar(L::B_KF + slot), ph, abort_flag))) break;
+          if (!(alive = wwait(L::B_KF + slot, ph))) break;
           tc_fence_after();
           const uint64_t kd = dk + uint32_t(slot * (L::TILE >> 4));
           if (tile_has(w.tile[0], j)) {
             issue_qk<D>(dS0, dq0, kd);
-            tc_commit(bar(L::B_SF + 0));
+            commit(L::B_SF + 0);
           }
           if (it > 0) {
             if (tile_has(w.tile[1], prev_j) && !(alive = pv_tile(1, prev_slot))) break;
-            tc_commit(bar(L::B_VE + prev_slot));
+            commit(L::B_VE + prev_slot);
           }
           if (tile_has(w.tile[1], j)) {
             issue_qk<D>(dS1, dq1, kd);
-            tc_commit(bar(L::B_SF + 1));
+            commit(L::B_SF + 1);
           }
-          tc_commit(bar(L::B_KE + slot));
-          if (it == w.U - 1) tc_commit(bar(L::B_QE));     // every Q.K^T of this item issued
-          if (!(alive = mbar_wait(bar(L::B_VF + slot), ph, abort_flag))) break;
+          commit(L::B_KE + slot);
+          if (it == w.U - 1) commit(L::B_QE);     // every Q.K^T of this item issued
+          if (!(alive = wwait(L::B_VF + slot, ph))) break;
           tc_fence_after();
           if (tile_has(w.tile[0], j) && !(alive = pv_tile(0, slot))) break;
           prev_j = j;
@@ -528,14 +537,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         }
         if (!alive) break;
         if (tile_has(w.tile[1], prev_j) && !(alive = pv_tile(1, prev_slot))) break;
-        tc_commit(bar(L::B_VE + prev_slot));
+        commit(L::B_VE + prev_slot);
         if (!first[0]) ++done[0];
         if (!first[1]) ++done[1];
         ++qi;
       }
       // drain: every issued tensor-core operation completes before teardown
-      tc_commit(bar(L::B_DRAIN));
+      commit(L::B_DRAIN);
       mbar_wait(bar(L::B_DRAIN), 0, nullptr);
+      __syncwarp();
     }
     __syncwarp();
   } else if (warp == 9) {
