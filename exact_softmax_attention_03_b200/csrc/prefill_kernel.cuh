@@ -109,7 +109,7 @@ static_assert(kFwdRegsLaunchMin <= kFwdRegsLaunch, "register split exceeds the l
 // Every kPolyEvery-th pair of exponentials in an unmasked score tile is
 // computed on the FMA pipe instead of the MUFU unit.
 #ifndef ATTN_POLY_EVERY
-#define ATTN_POLY_EVERY 4
+#define ATTN_POLY_EVERY 8
 #endif
 constexpr int kPolyEvery = ATTN_POLY_EVERY;
 
@@ -300,12 +300,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       float l = 0.f;                        // running sum of exp2((s - m) * c2)
       int n_in_item = 0;
       for (int j = T.bhi - 1; j >= T.blo; --j) {
-        bool wt = mbar_wait<1>(bar(L::B_SF + t), uint32_t(count & 1), abort_flag);
-        // the previous P.V of this item must be done before P is overwritten
-        // and before O is rescaled (at an item's first tile it was waited for
-        // in the previous epilogue)
-        if (wt && n_in_item > 0)
-          wt = mbar_wait<1>(bar(L::B_OD + t), uint32_t((count - 1) & 1), abort_flag);
+        // S_t(j) is issued after this tile's previous P.V and its commit covers
+        // every earlier MMA of the issuer, so once S is ready the previous P.V
+        // has completed: P may be overwritten and O rescaled.
+        const bool wt = mbar_wait<1>(bar(L::B_SF + t), uint32_t(count & 1), abort_flag);
         if (!__all_sync(0xffffffffu, wt)) { ok = false; break; }
         tc_fence_after();
 
