@@ -83,6 +83,34 @@ def make_for(w: Workload, seed: int = SEED_Q):
     return make_qkv(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, seed)
 
 
+def make_paged(k_cache, v_cache, page_size: int, seed: int = SEED_Q + 11, extra_pages: int = 3):
+    """Scatter contiguous caches ``[B, Lmax, Hkv, d]`` into shuffled page pools.
+
+    Returns ``(k_pages, v_pages, block_table)``: pools ``[num_pages, page_size,
+    Hkv, d]`` (bf16, CPU) holding every ``page_size`` keys of every sequence in
+    a page chosen by a seeded permutation, plus ``extra_pages`` pages of noise
+    that no table entry names, and ``block_table [B, Lmax // page_size]``
+    (int32) with ``block_table[b, i]`` = the page of keys
+    ``[i * page_size, (i + 1) * page_size)`` of sequence ``b``. ``Lmax`` must be
+    a multiple of ``page_size``.
+    """
+    B, Lmax, Hkv, d = k_cache.shape
+    if Lmax % page_size:
+        raise ValueError("Lmax must be a multiple of page_size")
+    per_seq = Lmax // page_size
+    num_pages = B * per_seq + extra_pages
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    perm = torch.randperm(num_pages, generator=g)[: B * per_seq]
+    block_table = perm.reshape(B, per_seq).to(torch.int32).contiguous()
+    k_pages = _randn((num_pages, page_size, Hkv, d), seed + 1)
+    v_pages = _randn((num_pages, page_size, Hkv, d), seed + 2)
+    idx = block_table.reshape(-1).long()
+    k_pages[idx] = k_cache.reshape(B * per_seq, page_size, Hkv, d)
+    v_pages[idx] = v_cache.reshape(B * per_seq, page_size, Hkv, d)
+    return k_pages.contiguous(), v_pages.contiguous(), block_table
+
+
 def ragged_seqlens(B: int, Lmax: int, seed: int = SEED_Q + 7) -> torch.Tensor:
     """int32 ``[B]`` cache lengths in ``[1, Lmax]`` (a mix of short and full rows)."""
     g = torch.Generator(device="cpu")

@@ -48,6 +48,8 @@ KERNEL_SOURCES = {
                         for f in ("sm100_ptx.cuh", "prefill_kernel.cuh")],
     "decode": ["exact_softmax_attention_03_b200/csrc/" + f
                for f in ("sm100_ptx.cuh", "decode_kernels.cuh")],
+    "decode_paged": ["exact_softmax_attention_03_b200/csrc/" + f
+                     for f in ("sm100_ptx.cuh", "decode_kernels.cuh")],
 }
 
 
@@ -64,6 +66,8 @@ def parse_args():
                     help="override the prefill batch (profiling a smaller case only)")
     ap.add_argument("--decode-batch", type=int, default=0,
                     help="override the decode batch (profiling a smaller case only)")
+    ap.add_argument("--page-size", type=int, default=16,
+                    help="keys per page in the paged-cache decode leg (16, 32, 64 or k*128)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -394,6 +398,31 @@ def run_ours(args, world, rank, local):
     d_all = metrics.decode_bytes(dw.B, dw.Hq, dw.Hkv, [dw.Nk] * dw.B, dw.d)
     d_value = whole_job_rate(kv_bytes, dms_max, world) / 1e9
 
+    # paged decode leg: the same logical cache scattered into shuffled pages of
+    # args.page_size keys (a seeded permutation; unused pool pages are never read)
+    ps = args.page_size
+    per_seq = dw.Nk // ps
+    n_pages = dw.B * per_seq + 64
+    gperm = torch.Generator(device="cpu")
+    gperm.manual_seed(shard_seed(rank) + 11)
+    perm = torch.randperm(n_pages, generator=gperm)[: dw.B * per_seq]
+    bt = perm.reshape(dw.B, per_seq).to(torch.int32).to(dev)
+    kpg = torch.empty((n_pages, ps, dw.Hkv, dw.d), dtype=torch.bfloat16, device=dev)
+    vpg = torch.empty_like(kpg)
+    kpg[perm.to(dev)] = kc.reshape(dw.B * per_seq, ps, dw.Hkv, dw.d)
+    vpg[perm.to(dev)] = vc.reshape(dw.B * per_seq, ps, dw.Hkv, dw.d)
+    del kc, vc
+
+    def dec_paged():
+        ea.attn_decode_paged(qd, kpg, vpg, bt, o=od, lse=lsed, num_splits=args.decode_splits,
+                             workspace=ws)
+
+    ptimes, plaunches = timed_kernel_loop(dec_paged, args.steps, args.warmup, world, None, None)
+    pms = statistics.mean(ptimes)
+    pms_max = max_over_ranks(pms, world)
+    p_value = whole_job_rate(kv_bytes, pms_max, world) / 1e9
+    del kpg, vpg
+
     # end-to-end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
@@ -457,6 +486,18 @@ def run_ours(args, world, rank, local):
                          "algorithmic_bytes": d_all,
                          "traffic": recorded_traffic("decode", "decode")},
             "gpu_launches": dlaunches,
+        },
+        "decode_paged": {
+            "workload": f"{dw.name}, paged cache ({ps}-key pages, shuffled pool)", "page_size": ps,
+            "value": p_value, "unit": "GB/s", "ms_per_step": pms_max,
+            "roofline": {"bound": "hbm", "achieved": kv_bytes / (pms * 1e-3) / 1e9,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": kv_bytes / (pms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                         "peak_source": f"{peak_src} hbm_gbs",
+                         "kernel": "decode_split_kernel<128,4,paged> + decode_combine_kernel<128>",
+                         "algorithmic_bytes": d_all,
+                         "traffic": recorded_traffic("decode_paged", f"decode_p{ps}")},
+            "gpu_launches": plaunches,
         },
         "clocks": clocks,
         "gpu_launches": launches,

@@ -19,8 +19,8 @@ import torch
 
 from ._lib import AttnError, check, load  # noqa: F401
 
-__all__ = ["attn_fwd", "attn_fwd_f32o", "attn_decode", "attn_decode_workspace_bytes",
-           "attn_decode_noalloc",
+__all__ = ["attn_fwd", "attn_fwd_f32o", "attn_decode", "attn_decode_paged",
+           "attn_decode_workspace_bytes", "attn_decode_noalloc",
            "attn_device_status", "attn_last_error", "attn_launch_count", "AttnError"]
 
 
@@ -122,6 +122,52 @@ def attn_decode(q, k_cache, v_cache, o=None, lse=None, seqlens=None, window_left
                              seqlens.data_ptr() if seqlens is not None else None,
                              B, Hq, Hkv, Lmax, d, float(scale), int(window_left), int(num_splits),
                              workspace.data_ptr(), ws_bytes, _stream_handle(stream)))
+    return o, lse
+
+
+def attn_decode_paged(q, k_pages, v_pages, block_table, o=None, lse=None, seqlens=None,
+                      window_left=-1, scale=None, num_splits=0, workspace=None, stream=None):
+    """Single-query decode over a paged KV cache. Returns ``(o, lse)``.
+
+    ``k_pages``/``v_pages`` are ``[num_pages, page_size, Hkv, d]`` bf16 pools;
+    ``block_table`` is ``[B, pages_per_seq]`` int32 on the device: logical key
+    ``t`` of sequence ``b`` lives at row ``t % page_size`` of page
+    ``block_table[b, t // page_size]``. Everything else is as in
+    :func:`attn_decode` with ``Lmax = pages_per_seq * page_size``.
+    """
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k_pages, "k_pages", torch.bfloat16, 4)
+    _need(v_pages, "v_pages", torch.bfloat16, 4)
+    _need(block_table, "block_table", torch.int32, 2)
+    B, Hq, d = q.shape
+    num_pages, page_size, Hkv, _ = k_pages.shape
+    if k_pages.shape[3] != d or v_pages.shape != k_pages.shape:
+        raise ValueError("page pools must be [num_pages, page_size, Hkv, d] matching q")
+    if block_table.shape[0] != B:
+        raise ValueError("block_table must be [B, pages_per_seq]")
+    pages_per_seq = block_table.shape[1]
+    if o is None:
+        o = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q.device)
+    _need(o, "o", torch.bfloat16, 3)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, 2)
+    if seqlens is not None:
+        _need(seqlens, "seqlens", torch.int32, 1)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    need = attn_decode_workspace_bytes(B, Hq, d, num_splits, pages_per_seq * page_size)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if not workspace.is_cuda:
+        raise ValueError("workspace must be a CUDA tensor")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    check(load().attn_decode_paged(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(), o.data_ptr(),
+                                   lse.data_ptr() if lse is not None else None,
+                                   block_table.data_ptr(),
+                                   seqlens.data_ptr() if seqlens is not None else None,
+                                   B, Hq, Hkv, num_pages, page_size, pages_per_seq, d, float(scale),
+                                   int(window_left), int(num_splits), workspace.data_ptr(), ws_bytes,
+                                   _stream_handle(stream)))
     return o, lse
 
 

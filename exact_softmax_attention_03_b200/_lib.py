@@ -40,6 +40,8 @@ SIGNATURES = {
                          ctypes.c_size_t, _vp]),
     "attn_decode_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _i,
                                  _vp]),
+    "attn_decode_paged": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
+                               _f, _i, _i, _vp, ctypes.c_size_t, _vp]),
     "attn_last_error": (ctypes.c_char_p, []),
     "attn_device_status": (_i, [_vp]),
     "attn_selftest_wait_timeout": (_i, [_vp]),

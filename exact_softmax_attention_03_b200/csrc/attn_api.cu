@@ -91,12 +91,14 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 // 4-D view {d, H, N, B} of a contiguous bf16 [B, N, H, d] tensor; box
 // {64, 1, 128, 1} with 128-byte swizzle (one 128-row x 128-byte block).
-int make_map(CUtensorMap* map, const void* base, int d, int H, int N, int B) {
+// 4-D view {d, H, N, B} of a [B, N, H, d] bf16 tensor, boxes of 64 columns x
+// box_rows rows with the 128-byte swizzle.
+int make_map(CUtensorMap* map, const void* base, int d, int H, int N, int B, int box_rows = 128) {
   auto enc = tensor_map_encoder();
   if (enc == nullptr) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   cuuint64_t dims[4] = {cuuint64_t(d), cuuint64_t(H), cuuint64_t(N), cuuint64_t(B)};
   cuuint64_t strides[3] = {cuuint64_t(d) * 2, cuuint64_t(H) * d * 2, cuuint64_t(N) * H * d * 2};
-  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t box[4] = {64, 1, cuuint32_t(box_rows), 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -250,14 +252,20 @@ DecodeShape decode_shape(int B, int Hq, int d, int num_splits, int Lmax) {
   return s;
 }
 
-template <int D, int GT>
+template <int D, int GT, bool PAGED>
 int launch_decode_kernels(attn::DecodeParams& p, const void* k_cache, const void* v_cache,
                           cudaStream_t stream, int dev) {
   using L = attn::DecLayout<D>;
   CUtensorMap mk, mv;
   int rc;
-  if ((rc = make_map(&mk, k_cache, D, p.Hkv, p.Lmax, p.B)) != ATTN_OK) return rc;
-  if ((rc = make_map(&mv, v_cache, D, p.Hkv, p.Lmax, p.B)) != ATTN_OK) return rc;
+  if constexpr (PAGED) {
+    const int rows = p.page_size < 128 ? p.page_size : 128;
+    if ((rc = make_map(&mk, k_cache, D, p.Hkv, p.page_size, p.num_pages, rows)) != ATTN_OK) return rc;
+    if ((rc = make_map(&mv, v_cache, D, p.Hkv, p.page_size, p.num_pages, rows)) != ATTN_OK) return rc;
+  } else {
+    if ((rc = make_map(&mk, k_cache, D, p.Hkv, p.Lmax, p.B)) != ATTN_OK) return rc;
+    if ((rc = make_map(&mv, v_cache, D, p.Hkv, p.Lmax, p.B)) != ATTN_OK) return rc;
+  }
   const int G = p.Hq / p.Hkv;
   const long long items = static_cast<long long>(p.B) * p.Hkv * (G / GT) * p.S;
   if (items > kMaxIndex) return fail(ATTN_ERR_INVALID_ARG, "decode problem too large");
@@ -267,16 +275,31 @@ int launch_decode_kernels(attn::DecodeParams& p, const void* k_cache, const void
   static std::atomic<unsigned long long> attr_set{0};   // per-device bit
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(attr_set.load() & bit)) {
-    cudaError_t e = cudaFuncSetAttribute(attn::decode_split_kernel<D, GT>,
+    cudaError_t e = cudaFuncSetAttribute(attn::decode_split_kernel<D, GT, PAGED>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_ALLOC);
     if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     attr_set.fetch_or(bit);
   }
   const int grid = static_cast<int>(std::min<long long>(items, sms));
-  attn::decode_split_kernel<D, GT><<<grid, attn::kDecodeSplitThreads, L::SMEM_ALLOC, stream>>>(mk, mv, p);
+  attn::decode_split_kernel<D, GT, PAGED><<<grid, attn::kDecodeSplitThreads, L::SMEM_ALLOC, stream>>>(mk, mv, p);
   const int n = p.B * p.Hq;
   attn::decode_combine_kernel<D><<<(n + 3) / 4, 128, 0, stream>>>(p);
   return ATTN_OK;
+}
+
+// Head dim and group tile are compile-time in the kernels: pick the instance.
+template <bool PAGED>
+int dispatch_decode(attn::DecodeParams& p, int d, const void* k_cache, const void* v_cache,
+                    cudaStream_t stream, int dev) {
+  const int GT = decode_group_tile(p.Hq / p.Hkv);
+  if (d == 128) {
+    if (GT == 4) return launch_decode_kernels<128, 4, PAGED>(p, k_cache, v_cache, stream, dev);
+    if (GT == 2) return launch_decode_kernels<128, 2, PAGED>(p, k_cache, v_cache, stream, dev);
+    return launch_decode_kernels<128, 1, PAGED>(p, k_cache, v_cache, stream, dev);
+  }
+  if (GT == 4) return launch_decode_kernels<64, 4, PAGED>(p, k_cache, v_cache, stream, dev);
+  if (GT == 2) return launch_decode_kernels<64, 2, PAGED>(p, k_cache, v_cache, stream, dev);
+  return launch_decode_kernels<64, 1, PAGED>(p, k_cache, v_cache, stream, dev);
 }
 
 // ------------------------------------------------------ no-alloc decode --
@@ -351,16 +374,7 @@ int attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
   p.chunk = sh.chunk;
   p.window_left = window_left < 0 ? -1 : window_left;
   p.scale_log2 = scale * 1.4426950408889634f;
-  const int GT = decode_group_tile(Hq / Hkv);
-  if (d == 128) {
-    if (GT == 4) rc = launch_decode_kernels<128, 4>(p, k_cache, v_cache, stream, dev);
-    else if (GT == 2) rc = launch_decode_kernels<128, 2>(p, k_cache, v_cache, stream, dev);
-    else rc = launch_decode_kernels<128, 1>(p, k_cache, v_cache, stream, dev);
-  } else {
-    if (GT == 4) rc = launch_decode_kernels<64, 4>(p, k_cache, v_cache, stream, dev);
-    else if (GT == 2) rc = launch_decode_kernels<64, 2>(p, k_cache, v_cache, stream, dev);
-    else rc = launch_decode_kernels<64, 1>(p, k_cache, v_cache, stream, dev);
-  }
+  rc = dispatch_decode<false>(p, d, k_cache, v_cache, stream, dev);
   if (rc != ATTN_OK) return rc;
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "attn_decode_noalloc launch: %s", cudaGetErrorString(e));
@@ -427,19 +441,69 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache, void* o
   p.chunk = sh.chunk;
   p.window_left = window_left < 0 ? -1 : window_left;
   p.scale_log2 = scale * 1.4426950408889634f;
-  const int GT = decode_group_tile(Hq / Hkv);
-  if (d == 128) {
-    if (GT == 4) rc = launch_decode_kernels<128, 4>(p, k_cache, v_cache, stream, dev);
-    else if (GT == 2) rc = launch_decode_kernels<128, 2>(p, k_cache, v_cache, stream, dev);
-    else rc = launch_decode_kernels<128, 1>(p, k_cache, v_cache, stream, dev);
-  } else {
-    if (GT == 4) rc = launch_decode_kernels<64, 4>(p, k_cache, v_cache, stream, dev);
-    else if (GT == 2) rc = launch_decode_kernels<64, 2>(p, k_cache, v_cache, stream, dev);
-    else rc = launch_decode_kernels<64, 1>(p, k_cache, v_cache, stream, dev);
-  }
+  rc = dispatch_decode<false>(p, d, k_cache, v_cache, stream, dev);
   if (rc != ATTN_OK) return rc;
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "attn_decode launch: %s", cudaGetErrorString(e));
+  g_launches.fetch_add(2);
+  return ok();
+}
+
+int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, void* o, float* lse,
+                      const int* block_table, const int* seqlens, int B, int Hq, int Hkv,
+                      int num_pages, int page_size, int pages_per_seq, int d, float scale,
+                      int window_left, int num_splits, void* workspace, size_t workspace_bytes,
+                      cudaStream_t stream) {
+  if (!q || !k_pages || !v_pages || !o || !block_table)
+    return fail(ATTN_ERR_INVALID_ARG, "q, k_pages, v_pages, o and block_table must be non-null");
+  if (B < 1 || Hq < 1 || Hkv < 1 || num_pages < 1 || pages_per_seq < 1)
+    return fail(ATTN_ERR_INVALID_ARG, "B, Hq, Hkv, num_pages, pages_per_seq must be >= 1");
+  if (!(page_size == 16 || page_size == 32 || page_size == 64 || (page_size >= 128 && page_size % 128 == 0)))
+    return fail(ATTN_ERR_INVALID_ARG, "page_size %d must be 16, 32, 64 or a multiple of 128", page_size);
+  if (Hq % Hkv != 0) return fail(ATTN_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
+  if (d != 64 && d != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim %d not in {64, 128}", d);
+  if (!finite_pos(scale)) return fail(ATTN_ERR_INVALID_ARG, "scale must be finite and > 0");
+  if (num_splits < 0) return fail(ATTN_ERR_INVALID_ARG, "num_splits must be >= 0");
+  if (!aligned(q, 16) || !aligned(k_pages, 16) || !aligned(v_pages, 16) || !aligned(o, 16))
+    return fail(ATTN_ERR_INVALID_ARG, "q, k_pages, v_pages, o must be 16-byte aligned");
+  if (!aligned(block_table, 4)) return fail(ATTN_ERR_INVALID_ARG, "block_table must be 4-byte aligned");
+  if (lse && !aligned(lse, 4)) return fail(ATTN_ERR_INVALID_ARG, "lse must be 4-byte aligned");
+  if (seqlens && !aligned(seqlens, 4)) return fail(ATTN_ERR_INVALID_ARG, "seqlens must be 4-byte aligned");
+  const long long Lmax = static_cast<long long>(pages_per_seq) * page_size;
+  if (Lmax > kMaxIndex || static_cast<long long>(B) * pages_per_seq > kMaxIndex ||
+      static_cast<long long>(B) * Hq > kMaxIndex || static_cast<long long>(num_pages) >= kMaxIndex)
+    return fail(ATTN_ERR_INVALID_ARG, "sizes too large");
+  const DecodeShape sh = decode_shape(B, Hq, d, num_splits, static_cast<int>(Lmax));
+  if (workspace == nullptr || workspace_bytes < sh.total)
+    return fail(ATTN_ERR_WORKSPACE, "workspace of %zu bytes needed, got %zu", sh.total,
+                workspace == nullptr ? size_t(0) : workspace_bytes);
+  if (!aligned(workspace, 256)) return fail(ATTN_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  int dev = 0;
+  int rc = check_device(&dev);
+  if (rc != ATTN_OK) return rc;
+
+  attn::DecodeParams p{};
+  p.q = static_cast<const uint16_t*>(q);
+  p.k = static_cast<const uint16_t*>(k_pages);
+  p.v = static_cast<const uint16_t*>(v_pages);
+  p.o = static_cast<uint16_t*>(o);
+  p.lse = lse;
+  p.seqlens = seqlens;
+  p.ws_acc = static_cast<float*>(workspace);
+  p.ws_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) + sh.acc_bytes);
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Lmax = static_cast<int>(Lmax);
+  p.S = sh.S;
+  p.chunk = sh.chunk;
+  p.window_left = window_left < 0 ? -1 : window_left;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.block_table = block_table;
+  p.page_size = page_size;
+  p.pages_per_seq = pages_per_seq;
+  p.num_pages = num_pages;
+  rc = dispatch_decode<true>(p, d, k_pages, v_pages, stream, dev);
+  if (rc != ATTN_OK) return rc;
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "attn_decode_paged launch: %s", cudaGetErrorString(e));
   g_launches.fetch_add(2);
   return ok();
 }

@@ -24,8 +24,8 @@ namespace attn {
 
 struct DecodeParams {
   const uint16_t* q;        // [B, Hq, D] bf16
-  const uint16_t* k;        // [B, Lmax, Hkv, D] bf16
-  const uint16_t* v;        // [B, Lmax, Hkv, D] bf16
+  const uint16_t* k;        // [B, Lmax, Hkv, D] bf16 (paged: [num_pages, page_size, Hkv, D])
+  const uint16_t* v;        // same layout as k
   uint16_t* o;              // [B, Hq, D] bf16
   float* lse;               // [B, Hq] or null
   const int* seqlens;       // [B] or null
@@ -35,6 +35,10 @@ struct DecodeParams {
   int window_left;
   float scale_log2;         // scale * log2(e)
   int n_items;              // B * Hkv * (G / GT) * S
+  // paged cache only: logical key t of sequence b is row t % page_size of page
+  // block_table[b * pages_per_seq + t / page_size]
+  const int* block_table;   // [B, pages_per_seq] int32
+  int page_size, pages_per_seq, num_pages;
 };
 
 
@@ -123,7 +127,13 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   return v;
 }
 
-template <int D, int GT>
+// PAGED: the K/V tensor maps view the page pool as [num_pages, page_size,
+// Hkv, D] with boxes of min(page_size, 128) rows; each 128-key tile is one box
+// per 64-column half (page_size a multiple of 128) or 128 / page_size boxes
+// (page_size 16, 32 or 64), each from the page the block table names. Pages
+// wholly past the visible keys are read at page index num_pages, outside the
+// map, which the copy engine fills with zeros (same byte count, no stale data).
+template <int D, int GT, bool PAGED>
 __global__ void __launch_bounds__(kDecodeSplitThreads, 1)
 decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const DecodeParams p) {
@@ -154,32 +164,62 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
   const int n_items = p.n_items;
   if (warp == 8) {
     // ======================= TMA producer ====================================
+    // The whole warp walks the stages (waits agree through a warp vote). Lane 0
+    // announces each stage's bytes; the copies are issued by lane 0 (contiguous
+    // cache) or, for a paged cache, by lane i for box i, in parallel.
     if (lane == 0) {
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      int st = 0;
-      bool alive = true;
-      for (int item = blockIdx.x; alive && item < n_items; item += gridDim.x) {
-        DecItem w;
-        dec_item<GT>(p, item, w);
-        for (int s = 0; s < w.n_stages; ++s, ++st) {
-          const int slot = st % L::STAGES;
-          const uint32_t ph = uint32_t(st / L::STAGES) & 1u;
-          if (!(alive = mbar_wait(bar(B_EMPTY + slot), ph ^ 1u, abort_flag))) break;
-          mbar_arrive_expect_tx(bar(B_FULL + slot), 2 * L::TILE);
-          const int key0 = w.k_first + 128 * s;
+    }
+    int st = 0;
+    bool alive = true;
+    // paged: this lane's box of the next stage has its page read from the block
+    // table one stage ahead, so the read overlaps the wait for a free slot
+    const int ps = PAGED ? p.page_size : 128;
+    const int rows = ps < 128 ? ps : 128;              // keys per box
+    const bool box_lane = PAGED && lane * rows < 128;
+    int page_next = 0;
+    auto fetch_page = [&](const DecItem& w, int s) -> int {
+      const int t = w.k_first + 128 * s + lane * rows;
+      return t < w.hi ? __ldg(p.block_table + size_t(w.b) * p.pages_per_seq + t / ps) : p.num_pages;
+    };
+    for (int item = blockIdx.x; alive && item < n_items; item += gridDim.x) {
+      DecItem w;
+      dec_item<GT>(p, item, w);
+      if (box_lane && w.n_stages > 0) page_next = fetch_page(w, 0);
+      for (int s = 0; s < w.n_stages; ++s, ++st) {
+        const int slot = st % L::STAGES;
+        const uint32_t ph = uint32_t(st / L::STAGES) & 1u;
+        const int page_cur = page_next;
+        if (box_lane && s + 1 < w.n_stages) page_next = fetch_page(w, s + 1);
+        if (!(alive = __all_sync(0xffffffffu, mbar_wait(bar(B_EMPTY + slot), ph ^ 1u, abort_flag))))
+          break;
+        if (lane == 0) mbar_arrive_expect_tx(bar(B_FULL + slot), 2 * L::TILE);
+        const int key0 = w.k_first + 128 * s;
+        if constexpr (!PAGED) {
+          if (lane == 0) {
+            for (int c = 0; c < D / 64; ++c) {
+              tma_load_4d(sb + L::OFF_K + slot * L::TILE + c * L::HALF, &tmK, bar(B_FULL + slot),
+                          c * 64, w.hkv, key0, w.b);
+              tma_load_4d(sb + L::OFF_V + slot * L::TILE + c * L::HALF, &tmV, bar(B_FULL + slot),
+                          c * 64, w.hkv, key0, w.b);
+            }
+          }
+        } else if (box_lane) {
+          const int r0 = lane * rows;
+          const int prow = (key0 + r0) % ps;
           for (int c = 0; c < D / 64; ++c) {
-            tma_load_4d(sb + L::OFF_K + slot * L::TILE + c * L::HALF, &tmK, bar(B_FULL + slot),
-                        c * 64, w.hkv, key0, w.b);
-            tma_load_4d(sb + L::OFF_V + slot * L::TILE + c * L::HALF, &tmV, bar(B_FULL + slot),
-                        c * 64, w.hkv, key0, w.b);
+            const uint32_t off = slot * L::TILE + c * L::HALF + r0 * 128;
+            tma_load_4d(sb + L::OFF_K + off, &tmK, bar(B_FULL + slot), c * 64, w.hkv, prow, page_cur);
+            tma_load_4d(sb + L::OFF_V + off, &tmV, bar(B_FULL + slot), c * 64, w.hkv, prow, page_cur);
           }
         }
+        __syncwarp();
       }
-      // no copy may still be landing at exit: wait for the last phase of each stage
-      for (int i = max(0, st - L::STAGES); i < st; ++i)
-        mbar_wait(bar(B_FULL + i % L::STAGES), uint32_t(i / L::STAGES) & 1u, nullptr);
     }
+    // no copy may still be landing at exit: wait for the last phase of each stage
+    for (int i = max(0, st - L::STAGES); i < st; ++i)
+      mbar_wait(bar(B_FULL + i % L::STAGES), uint32_t(i / L::STAGES) & 1u, nullptr);
     __syncwarp();
   } else {
     // ======================= consumer warps ==================================

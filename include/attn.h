@@ -110,6 +110,33 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache, void* o
                 void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * Single-query decode over a paged KV cache: the cache is split into
+ * fixed-size pages reached through a lookup table, so a sequence's keys need
+ * not be contiguous ("Inference Engineering", section 2.5 "Optimizing
+ * Attention", the PagedAttention paragraph). Logical key t of sequence b is
+ * row (t % page_size) of page block_table[b * pages_per_seq + t / page_size].
+ * Apart from where keys live, the operation, masks, splits and results are
+ * those of attn_decode with Lmax = pages_per_seq * page_size; for the same
+ * logical cache both return the same bits.
+ *   k_pages  : device, bf16 [num_pages, page_size, Hkv, d], 16-byte aligned;
+ *              v_pages likewise
+ *   block_table : device, int32 [B, pages_per_seq], 4-byte aligned; only the
+ *              entries covering keys [0, seqlens[b]) are read. An entry
+ *              outside [0, num_pages) reads zeros, never other memory.
+ *   page_size : 16, 32, 64, or a multiple of 128
+ *   num_pages, pages_per_seq >= 1
+ *   workspace : >= attn_decode_workspace_bytes(B, Hq, d, num_splits,
+ *              pages_per_seq * page_size) bytes, 256-byte aligned
+ *   q, o, lse, seqlens, window_left, num_splits : as attn_decode
+ * Returns ATTN_OK or an attn_status; nothing is launched on error.
+ */
+int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, void* o,
+                      float* lse, const int* block_table, const int* seqlens, int B, int Hq,
+                      int Hkv, int num_pages, int page_size, int pages_per_seq, int d,
+                      float scale, int window_left, int num_splits, void* workspace,
+                      size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * Decode without a workspace argument, for callers that cannot allocate
  * device memory. The pages have no counterpart to this; it exists for library
  * users only. Typical callers: a host program that owns every byte of device

@@ -14,7 +14,9 @@ from .attention import (  # noqa: F401
     oracle_attention,
     oracle_attention_rows,
     oracle_decode,
+    oracle_decode_paged,
     oracle_probabilities,
+    paged_to_contiguous,
     tiled_attention,
     online_softmax,
     merge_partials,

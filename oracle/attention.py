@@ -191,6 +191,41 @@ def oracle_decode(q, k_cache, v_cache, seqlens=None, window_left: int = -1,
     return O, LSE
 
 
+def paged_to_contiguous(pages, block_table, seqlens=None):
+    """Logical per-sequence cache from a paged pool.
+
+    "Inference Engineering", section 2.5 "Optimizing Attention" (the
+    PagedAttention paragraph): the cache is split into pages found through a
+    lookup table. Logical key ``t`` of sequence ``b`` is row ``t % page_size``
+    of page ``block_table[b, t // page_size]``. ``pages [num_pages, page_size,
+    Hkv, d]``, ``block_table [B, pages_per_seq]``; keys at or past ``seqlens[b]``
+    are left zero and their table entries are not read.
+    Returns ``[B, pages_per_seq * page_size, Hkv, d]`` (fp64).
+    """
+    bt = np.asarray(block_table, dtype=np.int64)
+    num_pages, ps, Hkv, d = pages.shape
+    B, per_seq = bt.shape
+    Lmax = per_seq * ps
+    if seqlens is None:
+        seqlens = [Lmax] * B
+    seqlens = [int(s) for s in np.asarray(seqlens).reshape(-1)]
+    out = np.zeros((B, Lmax, Hkv, d))
+    for b in range(B):
+        for t in range(min(seqlens[b], Lmax)):
+            page = int(bt[b, t // ps])
+            out[b, t] = _f64(pages[page, t % ps])      # one key row at a time
+    return out
+
+
+def oracle_decode_paged(q, k_pages, v_pages, block_table, seqlens=None, window_left: int = -1,
+                        scale: float | None = None):
+    """Decode over a paged cache: the plain decode of the logical cache that
+    the block table describes (``paged_to_contiguous``). Returns ``(O, LSE)``."""
+    kc = paged_to_contiguous(k_pages, block_table, seqlens)
+    vc = paged_to_contiguous(v_pages, block_table, seqlens)
+    return oracle_decode(q, kc, vc, seqlens, window_left=window_left, scale=scale)
+
+
 # ---------------------------------------------------------------------------
 # Second, independent formulations used only to check the one above.
 # ---------------------------------------------------------------------------

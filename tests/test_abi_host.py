@@ -33,7 +33,8 @@ def header_functions():
 def test_header_declares_the_expected_entry_points():
     assert header_functions() == sorted([
         "attn_fwd", "attn_fwd_f32o", "attn_decode_workspace_bytes", "attn_decode",
-        "attn_decode_noalloc", "attn_last_error", "attn_device_status", "attn_launch_count",
+        "attn_decode_paged", "attn_decode_noalloc", "attn_last_error", "attn_device_status",
+        "attn_launch_count",
         "attn_selftest_wait_timeout"])
 
 
@@ -119,6 +120,44 @@ def test_decode_rejects_bad_arguments_without_launch(lib, over, code):
     assert lib.attn_launch_count() == before
 
 
+def paged_args(**over):
+    a = dict(q=P, k=P, v=P, o=P, lse=None, bt=P, seqlens=None, B=2, Hq=8, Hkv=2, num_pages=40,
+             page_size=16, pages_per_seq=20, d=128, scale=0.1, window_left=-1, num_splits=0,
+             ws=P, ws_bytes=1 << 30, stream=None)
+    a.update(over)
+    return [a[k] for k in ("q", "k", "v", "o", "lse", "bt", "seqlens", "B", "Hq", "Hkv",
+                           "num_pages", "page_size", "pages_per_seq", "d", "scale", "window_left",
+                           "num_splits", "ws", "ws_bytes", "stream")]
+
+
+BAD_PAGED = [
+    (dict(bt=None), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(bt=P + 2), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(k=None), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(page_size=8), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(page_size=48), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(page_size=192), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(num_pages=0), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(pages_per_seq=0), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(Hq=6, Hkv=4), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(d=96), _lib.ATTN_ERR_UNSUPPORTED),
+    (dict(scale=float("nan")), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(pages_per_seq=1 << 27, page_size=256), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(ws=None), _lib.ATTN_ERR_WORKSPACE),
+    (dict(ws_bytes=100), _lib.ATTN_ERR_WORKSPACE),
+    (dict(ws=P + 16), _lib.ATTN_ERR_INVALID_ARG),
+]
+
+
+@pytest.mark.parametrize("over,code", BAD_PAGED)
+def test_paged_decode_rejects_bad_arguments_without_launch(lib, over, code):
+    before = lib.attn_launch_count()
+    rc = lib.attn_decode_paged(*paged_args(**over))
+    assert rc == code, lib.attn_last_error()
+    assert lib.attn_last_error()
+    assert lib.attn_launch_count() == before
+
+
 def test_workspace_bytes(lib):
     f = lib.attn_decode_workspace_bytes
     assert f(0, 8, 128, 0, 100) == 0
@@ -145,6 +184,9 @@ def test_binding_refuses_cpu_tensors():
         ea.attn_fwd(q, q, q)
     with pytest.raises(ValueError, match="CUDA"):
         ea.attn_decode(torch.zeros(1, 2, 64, dtype=torch.bfloat16), q, q)
+    with pytest.raises(ValueError, match="CUDA"):
+        ea.attn_decode_paged(torch.zeros(1, 2, 64, dtype=torch.bfloat16), q, q,
+                             torch.zeros(1, 4, dtype=torch.int32))
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
