@@ -83,6 +83,36 @@ def make_for(w: Workload, seed: int = SEED_Q):
     return make_qkv(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, seed)
 
 
+def varlen_lengths(n: int, lo: int, hi: int, seed: int = SEED_Q + 13) -> list:
+    """``n`` sequence lengths drawn uniformly from ``[lo, hi]`` (seeded)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    return [int(x) for x in torch.randint(lo, hi + 1, (n,), generator=g)]
+
+
+def make_varlen(lens_q, lens_k, Hq, Hkv, d, seed: int = SEED_Q, q_offset: int = 0,
+                tail: int = 0):
+    """Packed bf16 CPU tensors for sequences of the given query/key lengths.
+
+    Returns ``(q [total_q, Hq, d], k, v [total_k, Hkv, d], cu_q, cu_k)`` with
+    ``cu_*`` int32 ``[B + 1]`` offsets; the first sequence starts at row
+    ``q_offset`` of ``q`` and ``tail`` extra rows follow the last one (rows
+    that belong to no sequence).
+    """
+    cu_q = [q_offset]
+    for n in lens_q:
+        cu_q.append(cu_q[-1] + int(n))
+    cu_k = [0]
+    for n in lens_k:
+        cu_k.append(cu_k[-1] + int(n))
+    total_q = cu_q[-1] + tail
+    total_k = max(cu_k[-1], 1)
+    q = _randn((total_q, Hq, d), seed)
+    k = _randn((total_k, Hkv, d), seed + 1)
+    v = _randn((total_k, Hkv, d), seed + 2)
+    return (q, k, v, torch.tensor(cu_q, dtype=torch.int32), torch.tensor(cu_k, dtype=torch.int32))
+
+
 def make_paged(k_cache, v_cache, page_size: int, seed: int = SEED_Q + 11, extra_pages: int = 3):
     """Scatter contiguous caches ``[B, Lmax, Hkv, d]`` into shuffled page pools.
 

@@ -376,6 +376,27 @@ def run_ours(args, world, rank, local):
     tiles = metrics.executed_tiles(w.Nq, w.Nk, w.causal, w.window_left) * w.B * w.Hq
     clocks = sampler.summary()
 
+    # packed variable-length prefill leg: 16 causal sequences with seeded
+    # lengths in [256, 4096], MHA H32 d128, no padding
+    vl_lens = ai.varlen_lengths(16, 256, 4096, seed=shard_seed(rank) + 13)
+    vq_h, vk_h, vv_h, vcq_h, vck_h = ai.make_varlen(vl_lens, vl_lens, 32, 32, 128,
+                                                   seed=shard_seed(rank) + 17)
+    vq, vk, vv, vcq, vck = (t.to(dev) for t in (vq_h, vk_h, vv_h, vcq_h, vck_h))
+    vo = torch.empty_like(vq)
+    vlse = torch.empty((32, vq.shape[0]), dtype=torch.float32, device=dev)
+    vmax = max(vl_lens)
+
+    def fwd_varlen():
+        ea.attn_fwd_varlen(vq, vk, vv, vcq, vck, vmax, vmax, o=vo, lse=vlse, causal=True)
+
+    vtimes, vlaunches = timed_kernel_loop(fwd_varlen, args.steps, args.warmup, world, flush, None)
+    vms = statistics.mean(vtimes)
+    vms_max = max_over_ranks(vms, world)
+    v_flops = sum(metrics.attn_flops(1, 32, n, n, 128, True, -1) for n in vl_lens)
+    v_value = whole_job_rate(v_flops, vms_max, world) / 1e12
+    v_achieved = v_flops / (vms * 1e-3) / 1e12
+    del vq, vk, vv, vo
+
     # decode leg
     dw = ai.GQA_DECODE
     if args.decode_batch:
@@ -486,6 +507,16 @@ def run_ours(args, world, rank, local):
                          "algorithmic_bytes": d_all,
                          "traffic": recorded_traffic("decode", "decode")},
             "gpu_launches": dlaunches,
+        },
+        "varlen": {
+            "workload": f"MHA causal packed prefill, 16 sequences of {min(vl_lens)}-{max(vl_lens)} "
+                        f"tokens ({sum(vl_lens)} total) H32 d128",
+            "value": v_value, "unit": "TFLOP/s", "ms_per_step": vms_max,
+            "roofline": {"bound": "tensor", "achieved": v_achieved, "peak": peak_t,
+                         "unit": "TFLOP/s", "frac": v_achieved / peak_t,
+                         "peak_source": f"{peak_src} bf16_tflops (burst)",
+                         "kernel": "attn_fwd_kernel<128,false> (packed)", "traffic": None},
+            "gpu_launches": vlaunches,
         },
         "decode_paged": {
             "workload": f"{dw.name}, paged cache ({ps}-key pages, shuffled pool)", "page_size": ps,

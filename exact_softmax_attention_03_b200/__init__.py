@@ -19,7 +19,7 @@ import torch
 
 from ._lib import AttnError, check, load  # noqa: F401
 
-__all__ = ["attn_fwd", "attn_fwd_f32o", "attn_decode", "attn_decode_paged",
+__all__ = ["attn_fwd", "attn_fwd_f32o", "attn_fwd_varlen", "attn_decode", "attn_decode_paged",
            "attn_decode_workspace_bytes", "attn_decode_noalloc",
            "attn_device_status", "attn_last_error", "attn_launch_count", "AttnError"]
 
@@ -81,6 +81,43 @@ def attn_fwd(q, k, v, o=None, lse=None, causal=False, window_left=-1, scale=None
 def attn_fwd_f32o(q, k, v, o=None, lse=None, causal=False, window_left=-1, scale=None, stream=None):
     """Forward attention, float32 output. Returns ``(o, lse)``."""
     return _fwd(q, k, v, o, lse, causal, window_left, scale, stream, True)
+
+
+def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, o=None,
+                    lse=None, causal=False, window_left=-1, scale=None, stream=None):
+    """Forward attention over packed variable-length sequences. Returns ``(o, lse)``.
+
+    ``q [total_q, Hq, d]``, ``k``/``v [total_k, Hkv, d]`` (bf16, CUDA);
+    ``cu_seqlens_q``/``cu_seqlens_k`` int32 ``[B + 1]`` on the device (sequence
+    ``b`` owns rows ``[cu[b], cu[b+1])``); ``max_seqlen_q``/``max_seqlen_k`` are
+    host ints bounding every sequence's length. ``lse`` is ``[Hq, total_q]``.
+    """
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k, "k", torch.bfloat16, 3)
+    _need(v, "v", torch.bfloat16, 3)
+    _need(cu_seqlens_q, "cu_seqlens_q", torch.int32, 1)
+    _need(cu_seqlens_k, "cu_seqlens_k", torch.int32, 1)
+    total_q, Hq, d = q.shape
+    total_k, Hkv, dk = k.shape
+    if dk != d or v.shape != k.shape:
+        raise ValueError("k and v must be [total_k, Hkv, d] matching q")
+    B = cu_seqlens_q.shape[0] - 1
+    if B < 1 or cu_seqlens_k.shape[0] != B + 1:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must both have B + 1 entries")
+    if o is None:
+        o = torch.empty((total_q, Hq, d), dtype=torch.bfloat16, device=q.device)
+    _need(o, "o", torch.bfloat16, 3)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, 2)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    check(load().attn_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                 lse.data_ptr() if lse is not None else None,
+                                 cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), B, Hq, Hkv,
+                                 total_q, total_k, int(max_seqlen_q), int(max_seqlen_k), d,
+                                 float(scale), int(bool(causal)), int(window_left),
+                                 _stream_handle(stream)))
+    return o, lse
 
 
 def attn_decode_workspace_bytes(B: int, Hq: int, d: int, num_splits: int = 0, Lmax: int = 1) -> int:

@@ -130,21 +130,36 @@ int validate_fwd(const void* q, const void* k, const void* v, const void* o, con
   return ATTN_OK;
 }
 
-template <int D, bool F32OUT>
+// Packed variable-length input: sequence offsets (device) and packed row counts.
+struct Packed {
+  const int* cu_q;
+  const int* cu_k;
+  int total_q, total_k;
+};
+
+template <int D, bool F32OUT, bool VARLEN>
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                int Hkv, int Nq, int Nk, float scale, int causal, int window_left,
-               cudaStream_t stream, int dev) {
+               cudaStream_t stream, int dev, const Packed* pk = nullptr) {
   using L = attn::FwdLayout<D>;
   CUtensorMap mq, mk, mv;
   int rc;
-  if ((rc = make_map(&mq, q, D, Hq, Nq, B)) != ATTN_OK) return rc;
-  if ((rc = make_map(&mk, k, D, Hkv, Nk, B)) != ATTN_OK) return rc;
-  if ((rc = make_map(&mv, v, D, Hkv, Nk, B)) != ATTN_OK) return rc;
+  // packed input: one "batch" of total rows; the kernel adds each sequence's offset
+  const int rq = pk ? pk->total_q : Nq, rk = pk ? pk->total_k : Nk, nb = pk ? 1 : B;
+  if ((rc = make_map(&mq, q, D, Hq, rq, nb)) != ATTN_OK) return rc;
+  if ((rc = make_map(&mk, k, D, Hkv, rk, nb)) != ATTN_OK) return rc;
+  if ((rc = make_map(&mv, v, D, Hkv, rk, nb)) != ATTN_OK) return rc;
 
   attn::FwdParams p{};
   p.o = o;
   p.lse = lse;
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Nq = Nq; p.Nk = Nk;
+  if (pk) {
+    p.cu_q = pk->cu_q;
+    p.cu_k = pk->cu_k;
+    p.total_q = pk->total_q;
+    p.total_k = pk->total_k;
+  }
   p.causal = causal;
   p.window_left = window_left < 0 ? -1 : window_left;
   p.scale = scale;
@@ -159,8 +174,12 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     p.n_units = (p.n_qblk + 1) / 2;
     p.n_bh = B * Hq;
   }
+  p.nbh_seq = p.n_bh / B;
   const long long items = static_cast<long long>(p.n_units) * p.n_bh;
   if (items > kMaxIndex) return fail(ATTN_ERR_INVALID_ARG, "problem too large for one launch");
+  if (pk && (B > L::VL_MAX_SEQS || p.n_units > L::VL_MAX_UNITS))
+    return fail(ATTN_ERR_INVALID_ARG, "packed input limited to %d sequences and %d row units "
+                "(max_seqlen_q %d gives %d)", L::VL_MAX_SEQS, L::VL_MAX_UNITS, Nq, p.n_units);
   p.n_items = static_cast<int>(items);
   int sms = 0;
   if ((rc = sm_count(dev, &sms)) != ATTN_OK) return rc;
@@ -171,17 +190,17 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   if (!(attr_set.load() & bit)) {
     // the in-kernel register split needs this many registers per thread at launch
     cudaFuncAttributes fa{};
-    cudaError_t e = cudaFuncGetAttributes(&fa, attn::attn_fwd_kernel<D, F32OUT>);
+    cudaError_t e = cudaFuncGetAttributes(&fa, attn::attn_fwd_kernel<D, F32OUT, VARLEN>);
     if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "cudaFuncGetAttributes: %s", cudaGetErrorString(e));
     if (fa.numRegs < attn::kFwdRegsLaunchMin)
       return fail(ATTN_ERR_UNSUPPORTED, "attn_fwd kernel built with %d registers per thread, needs %d",
                   fa.numRegs, attn::kFwdRegsLaunchMin);
-    e = cudaFuncSetAttribute(attn::attn_fwd_kernel<D, F32OUT>,
+    e = cudaFuncSetAttribute(attn::attn_fwd_kernel<D, F32OUT, VARLEN>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_ALLOC);
     if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     attr_set.fetch_or(bit);
   }
-  attn::attn_fwd_kernel<D, F32OUT><<<unsigned(grid), attn::kFwdThreads, L::SMEM_ALLOC, stream>>>(mq, mk, mv, p);
+  attn::attn_fwd_kernel<D, F32OUT, VARLEN><<<unsigned(grid), attn::kFwdThreads, L::SMEM_ALLOC, stream>>>(mq, mk, mv, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "attn_fwd launch: %s", cudaGetErrorString(e));
   g_launches.fetch_add(1);
@@ -190,17 +209,21 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
 
 int fwd_entry(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
               int Hkv, int Nq, int Nk, int d, float scale, int causal, int window_left,
-              cudaStream_t stream, bool f32out) {
+              cudaStream_t stream, bool f32out, const Packed* pk = nullptr) {
   int rc = validate_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal);
   if (rc != ATTN_OK) return rc;
   int dev = 0;
   if ((rc = check_device(&dev)) != ATTN_OK) return rc;
-  if (d == 128) {
-    return f32out ? launch_fwd<128, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, window_left, stream, dev)
-                  : launch_fwd<128, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, window_left, stream, dev);
+  if (pk != nullptr) {   // packed sequences: bf16 output only
+    return d == 128 ? launch_fwd<128, false, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, window_left, stream, dev, pk)
+                    : launch_fwd<64, false, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, window_left, stream, dev, pk);
   }
-  return f32out ? launch_fwd<64, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, window_left, stream, dev)
-                : launch_fwd<64, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, window_left, stream, dev);
+  if (d == 128) {
+    return f32out ? launch_fwd<128, true, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, window_left, stream, dev)
+                  : launch_fwd<128, false, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, window_left, stream, dev);
+  }
+  return f32out ? launch_fwd<64, true, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, window_left, stream, dev)
+                : launch_fwd<64, false, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, window_left, stream, dev);
 }
 
 // ------------------------------------------------------------------ decode --
@@ -395,6 +418,25 @@ int attn_fwd_f32o(const void* q, const void* k, const void* v, float* o, float* 
   return fwd_entry(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, window_left, stream, true);
 }
 
+int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                    const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int Hq, int Hkv,
+                    int total_q, int total_k, int max_seqlen_q, int max_seqlen_k, int d,
+                    float scale, int causal, int window_left, cudaStream_t stream) {
+  if (!cu_seqlens_q || !cu_seqlens_k)
+    return fail(ATTN_ERR_INVALID_ARG, "cu_seqlens_q and cu_seqlens_k must be non-null");
+  if (!aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4))
+    return fail(ATTN_ERR_INVALID_ARG, "cu_seqlens must be 4-byte aligned");
+  if (total_q < 1 || total_k < 1)
+    return fail(ATTN_ERR_INVALID_ARG, "total_q and total_k must be >= 1");
+  if (max_seqlen_q > total_q || max_seqlen_k > total_k)
+    return fail(ATTN_ERR_INVALID_ARG, "max_seqlen_q/k cannot exceed total_q/k");
+  if (static_cast<long long>(total_q) * Hq > kMaxIndex || static_cast<long long>(total_k) * Hkv > kMaxIndex)
+    return fail(ATTN_ERR_INVALID_ARG, "sizes too large");
+  const Packed pk{cu_seqlens_q, cu_seqlens_k, total_q, total_k};
+  return fwd_entry(q, k, v, o, lse, B, Hq, Hkv, max_seqlen_q, max_seqlen_k, d, scale, causal,
+                   window_left, stream, false, &pk);
+}
+
 size_t attn_decode_workspace_bytes(int B, int Hq, int d, int num_splits, int Lmax) {
   if (B < 1 || Hq < 1 || Lmax < 1 || (d != 64 && d != 128) || num_splits < 0) return 0;
   return decode_shape(B, Hq, d, num_splits, Lmax).total;
@@ -517,6 +559,9 @@ int attn_device_status(cudaStream_t stream) {
   e = cudaMemcpyFromSymbol(&val, attn::g_attn_status, sizeof(int));
   if (e == cudaSuccess) e = cudaMemcpyToSymbol(attn::g_attn_status, &zero, sizeof(int));
   if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "status word: %s", cudaGetErrorString(e));
+  if (val == attn::kStatusBadInput)
+    return fail(ATTN_ERR_INVALID_ARG, "a device-side check failed (inconsistent cu_seqlens): "
+                                      "the offending sequences were skipped");
   if (val != 0) return fail(ATTN_ERR_TIMEOUT, "a device-side wait timed out");
   return ok();
 }

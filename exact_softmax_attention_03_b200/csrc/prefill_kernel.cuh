@@ -40,6 +40,17 @@
 
 namespace attn {
 
+// Packed-sequence schedule tables in shared memory (ints): perm[kVlMaxSeqs]
+// (sequences sorted by row units, longest first), cnt[kVlMaxUnits + 1]
+// (cnt[u]: sequences with more than u units), lvl[kVlMaxUnits + 1] (first
+// item of unit level u), cur[kVlMaxUnits + 1] (scatter cursors).
+constexpr int kVlMaxSeqs = 2048;
+constexpr int kVlMaxUnits = 1024;
+constexpr int kVlCnt = kVlMaxSeqs;
+constexpr int kVlLvl = kVlCnt + kVlMaxUnits + 1;
+constexpr int kVlCur = kVlLvl + kVlMaxUnits + 1;
+constexpr int kVlInts = kVlCur + kVlMaxUnits + 1;
+
 template <int D>
 struct FwdLayout {
   static constexpr int BM = 128;                       // query rows per tile
@@ -64,8 +75,13 @@ struct FwdLayout {
   static constexpr int B_OE = B_OD + 2;                 // O read by the epilogue, + tile
   static constexpr int B_DRAIN = B_OE + 2;
   static constexpr int NBAR = B_DRAIN + 1;
-  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // [0] TMEM base, [1] abort flag
-  static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // [0] TMEM base, [1] abort flag, [2] items
+  // packed-sequence schedule: sequences sorted by row units (longest first),
+  // per-unit-level sequence counts, and the first item of each level
+  static constexpr int VL_MAX_SEQS = kVlMaxSeqs;
+  static constexpr int VL_MAX_UNITS = kVlMaxUnits;
+  static constexpr int OFF_VL = OFF_MISC + 16;                           // VarlenTables
+  static constexpr int BYTES = OFF_VL + 4 * kVlInts;
   static constexpr int SMEM_ALLOC = BYTES + 1024;       // slack for 1024-byte alignment
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
@@ -74,9 +90,15 @@ struct FwdLayout {
 };
 
 struct FwdParams {
-  void* o;                 // [B, Nq, Hq, D] bf16 or f32
-  float* lse;              // [B, Hq, Nq] or null
-  int B, Hq, Hkv, Nq, Nk;
+  void* o;                 // [B, Nq, Hq, D] bf16 or f32 (packed: [total_q, Hq, D])
+  float* lse;              // [B, Hq, Nq] or null (packed: [Hq, total_q])
+  int B, Hq, Hkv, Nq, Nk;  // packed: Nq, Nk are the longest sequence lengths
+  // Packed variable-length sequences (kernel built with VARLEN): sequence b owns
+  // query rows [cu_q[b], cu_q[b + 1]) of Q/O and keys [cu_k[b], cu_k[b + 1]) of K/V.
+  const int* cu_q;
+  const int* cu_k;
+  int total_q, total_k;
+  int nbh_seq;             // items per (sequence, row unit): n_bh / B
   int causal, window_left;
   float scale;             // softmax scale
   float scale_log2;        // scale * log2(e)
@@ -114,7 +136,8 @@ static_assert(kFwdRegsLaunchMin <= kFwdRegsLaunch, "register split exceeds the l
 constexpr int kPolyEvery = ATTN_POLY_EVERY;
 
 struct TileInfo {
-  int hq, row0, active;    // query head, first row, any row < Nq
+  int hq, row0, active;    // query head, first row, any row < nq
+  int nq, nk;              // query rows and keys of this tile's sequence
   int blo, bhi;            // key blocks [blo, bhi); empty if bhi <= blo
 };
 
@@ -122,10 +145,10 @@ __device__ __forceinline__ void tile_range(const FwdParams& p, TileInfo& t) {
   t.blo = 0;
   t.bhi = 0;
   if (!t.active) return;
-  const int r_last = min(t.row0 + 127, p.Nq - 1);
-  const int qf = t.row0 + p.Nk - p.Nq;
-  const int ql = r_last + p.Nk - p.Nq;
-  const int hi = p.causal ? min(p.Nk, ql + 1) : p.Nk;
+  const int r_last = min(t.row0 + 127, t.nq - 1);
+  const int qf = t.row0 + t.nk - t.nq;
+  const int ql = r_last + t.nk - t.nq;
+  const int hi = p.causal ? min(t.nk, ql + 1) : t.nk;
   const int lo = p.window_left >= 0 ? max(0, qf - p.window_left) : 0;
   if (hi <= lo) return;
   t.blo = lo / 128;
@@ -139,10 +162,10 @@ __device__ __forceinline__ bool tile_has(const TileInfo& t, int j) {
 // Whether key block j needs element-wise masking for this tile's rows.
 __device__ __forceinline__ bool block_needs_mask(const FwdParams& p, const TileInfo& t, int j) {
   const int kb0 = j * 128, kb1 = kb0 + 127;
-  const int r_last = min(t.row0 + 127, p.Nq - 1);
-  const int qf = t.row0 + p.Nk - p.Nq;
-  const int ql = r_last + p.Nk - p.Nq;
-  return kb1 >= p.Nk || (p.causal && kb1 > qf) || (p.window_left >= 0 && kb0 < ql - p.window_left);
+  const int r_last = min(t.row0 + 127, t.nq - 1);
+  const int qf = t.row0 + t.nk - t.nq;
+  const int ql = r_last + t.nk - t.nq;
+  return kb1 >= t.nk || (p.causal && kb1 > qf) || (p.window_left >= 0 && kb0 < ql - p.window_left);
 }
 
 // Both are called by the whole issuer warp (warp-uniform operands); one
@@ -177,13 +200,91 @@ __device__ __forceinline__ void issue_pv_half(uint32_t d_tmem, uint32_t p_tmem, 
 // One work item: a (batch, head-or-head-pair, row unit) and its two tiles.
 struct WorkItem {
   int b, hkv;
+  int q0, k0, bc;          // first Q row and first key of the sequence, batch coordinate
   TileInfo tile[2];
   int ubhi, U;             // key blocks visited: ubhi-1 down to ubhi-U
 };
 
-__device__ __forceinline__ void decode_item(const FwdParams& p, int item, WorkItem& w) {
-  const int unit = p.n_units - 1 - item / p.n_bh;        // longest rows first
-  const int bh = item % p.n_bh;
+// Packed sequences: the work list holds only the items that exist, longest
+// rows first. Sequences are sorted by their number of row units (descending),
+// so at unit level u the sequences with more than u units are a prefix
+// perm[0 .. cnt[u]) of the sorted order; level u's items start at lvl[u].
+
+__device__ __forceinline__ int varlen_valid_rows(const FwdParams& p, int b) {
+  const int q0 = __ldg(p.cu_q + b), q1 = __ldg(p.cu_q + b + 1);
+  const int k0 = __ldg(p.cu_k + b), k1 = __ldg(p.cu_k + b + 1);
+  const bool good = 0 <= q0 && q0 <= q1 && q1 <= p.total_q && q1 - q0 <= p.Nq &&
+                    0 <= k0 && k0 <= k1 && k1 <= p.total_k && k1 - k0 <= p.Nk;
+  return good ? q1 - q0 : -1;
+}
+
+__device__ __forceinline__ int varlen_units(const FwdParams& p, int nq) {
+  const int per_unit = p.pair_heads ? 1 : 2;             // 128-row blocks per unit
+  return nq <= 0 ? 0 : ((nq + 127) / 128 + per_unit - 1) / per_unit;
+}
+
+// Built by every thread of the CTA before the warp roles split (it ends with
+// a CTA barrier); every CTA builds the same lists. Sequences with inconsistent
+// offsets get no items and raise the status word.
+__device__ void build_varlen_sched(const FwdParams& p, int* vl, int* n_items) {
+  int* perm = vl;
+  int* cnt = vl + kVlCnt;
+  int* lvl = vl + kVlLvl;
+  int* cur = vl + kVlCur;
+  const int U = p.n_units;
+  const int nbh = p.nbh_seq;                             // items per (sequence, unit)
+  for (int u = threadIdx.x; u <= U; u += blockDim.x) cnt[u] = 0;
+  __syncthreads();
+  for (int b = threadIdx.x; b < p.B; b += blockDim.x) {
+    const int nq = varlen_valid_rows(p, b);
+    if (nq < 0) atomicExch(&g_attn_status, kStatusBadInput);
+    atomicAdd(&cnt[varlen_units(p, nq)], 1);             // histogram of unit counts
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // buckets laid out from U units down to 0: cnt[v] becomes the first slot of
+    // bucket v, which is also the number of sequences with more than v units
+    int slot = 0;
+    for (int v = U; v >= 0; --v) {
+      const int h = cnt[v];
+      cnt[v] = slot;
+      cur[v] = slot;
+      slot += h;
+    }
+    int item = 0;
+    for (int u = U - 1; u >= 0; --u) {
+      lvl[u] = item;
+      item += cnt[u] * nbh;
+    }
+    *n_items = item;
+  }
+  __syncthreads();
+  for (int b = threadIdx.x; b < p.B; b += blockDim.x)
+    perm[atomicAdd(&cur[varlen_units(p, varlen_valid_rows(p, b))], 1)] = b;
+  __syncthreads();
+}
+
+// vl: the packed-sequence tables (null for the closed-form work list).
+template <bool VARLEN>
+__device__ __forceinline__ void decode_item(const FwdParams& p, int item, WorkItem& w,
+                                            const int* vl) {
+  int unit, bh;
+  if constexpr (VARLEN) {
+    const int* lvl = vl + kVlLvl;
+    // level: the lowest u whose first item is <= item (lvl grows as u falls)
+    int lo = 0, hi = p.n_units - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (lvl[mid] <= item) hi = mid; else lo = mid + 1;
+    }
+    unit = lo;
+    const int r = item - lvl[unit];
+    const int s = r / p.nbh_seq;
+    bh = vl[s] * p.nbh_seq + (r - s * p.nbh_seq);
+  } else {
+    unit = p.n_units - 1 - item / p.n_bh;                // longest rows first
+    bh = item % p.n_bh;
+  }
   if (p.pair_heads) {
     const int G = p.Hq / p.Hkv;
     const int pairs = G / 2;
@@ -206,9 +307,30 @@ __device__ __forceinline__ void decode_item(const FwdParams& p, int item, WorkIt
       w.tile[t].row0 = (2 * unit + t) * 128;
     }
   }
+  int nq = p.Nq, nk = p.Nk;
+  w.q0 = 0;
+  w.k0 = 0;
+  w.bc = w.b;
+  if constexpr (VARLEN) {
+    // sequence bounds from the offsets; an inconsistent sequence (outside the
+    // packed tensors, or longer than the longest length the host gave) is
+    // skipped and flagged, so nothing is written outside O and LSE
+    const int q0 = __ldg(p.cu_q + w.b), q1 = __ldg(p.cu_q + w.b + 1);
+    const int k0 = __ldg(p.cu_k + w.b), k1 = __ldg(p.cu_k + w.b + 1);
+    const bool good = 0 <= q0 && q0 <= q1 && q1 <= p.total_q && q1 - q0 <= p.Nq &&
+                      0 <= k0 && k0 <= k1 && k1 <= p.total_k && k1 - k0 <= p.Nk;
+    if (!good) atomicExch(&g_attn_status, kStatusBadInput);
+    nq = good ? q1 - q0 : 0;
+    nk = good ? k1 - k0 : 0;
+    w.q0 = good ? q0 : 0;
+    w.k0 = good ? k0 : 0;
+    w.bc = 0;
+  }
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
-    w.tile[t].active = w.tile[t].row0 < p.Nq;
+    w.tile[t].nq = nq;
+    w.tile[t].nk = nk;
+    w.tile[t].active = w.tile[t].row0 < nq;
     tile_range(p, w.tile[t]);
   }
   const bool ne0 = w.tile[0].bhi > w.tile[0].blo, ne1 = w.tile[1].bhi > w.tile[1].blo;
@@ -223,14 +345,14 @@ __device__ __forceinline__ void decode_item(const FwdParams& p, int item, WorkIt
 
 // k-th work item of this CTA in a boustrophedon order over the items sorted
 // longest first (close to a longest-processing-time schedule); -1 when done.
-__device__ __forceinline__ int item_of(const FwdParams& p, int k) {
+__device__ __forceinline__ int item_of(int n_items, int k) {
   const int G = int(gridDim.x);
   const int c = (k & 1) ? (G - 1 - int(blockIdx.x)) : int(blockIdx.x);
   const long long i = static_cast<long long>(k) * G + c;
-  return i < p.n_items ? int(i) : -1;
+  return i < n_items ? int(i) : -1;
 }
 
-template <int D, bool F32OUT>
+template <int D, bool F32OUT, bool VARLEN>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -275,6 +397,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  // the work list: closed form, or the compact list of packed sequences
+  const int* vs = nullptr;
+  int n_items = p.n_items;
+  if constexpr (VARLEN) {
+    int* vl = reinterpret_cast<int*>(smem + L::OFF_VL);
+    int* vl_items = reinterpret_cast<int*>(smem + L::OFF_MISC + 8);
+    build_varlen_sched(p, vl, vl_items);
+    vs = vl;
+    n_items = *vl_items;
+  }
 
   if (warp < 8) {
     // ======================= softmax warpgroups ==============================
@@ -288,14 +420,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     int count = 0;                          // S tiles processed so far (all items)
     bool ok = true;
     for (int k = 0; ok; ++k) {
-      const int item = item_of(p, k);
+      const int item = item_of(n_items, k);
       if (item < 0) break;
       WorkItem w;
-      decode_item(p, item, w);
+      decode_item<VARLEN>(p, item, w, vs);
       const TileInfo T = t ? w.tile[1] : w.tile[0];   // by value: no local-memory copy of w
       if (!T.active) continue;
       const int r = T.row0 + row;
-      const int qpos = r + p.Nk - p.Nq;
+      const int qpos = r + T.nk - T.nq;
       float m = -CUDART_INF_F;              // running max (raw score units)
       float l = 0.f;                        // running sum of exp2((s - m) * c2)
       int n_in_item = 0;
@@ -319,7 +451,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (masked) {
           // allowed keys of this row, relative to the block: [lo_rel, hi_rel]
           const int kb0 = j * 128;
-          int hi = p.Nk - 1;
+          int hi = T.nk - 1;
           if (p.causal) hi = min(hi, qpos);
           int lo = 0;
           if (p.window_left >= 0) lo = qpos - p.window_left;
@@ -428,9 +560,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
         for (int e = 0; e < D; ++e) o[e] = 0u;
       }
-      if (r < p.Nq) {
+      if (r < T.nq) {
         const float inv = (l > 0.f) ? 1.f / l : 0.f;
-        const size_t obase = ((size_t(w.b) * p.Nq + r) * p.Hq + T.hq) * D;
+        const size_t orow = VARLEN ? size_t(w.q0) + r : size_t(w.b) * p.Nq + r;
+        const size_t obase = (orow * p.Hq + T.hq) * D;
         if constexpr (F32OUT) {
           float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + obase);
 #pragma unroll
@@ -450,7 +583,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           }
         }
         if (p.lse != nullptr)
-          p.lse[(size_t(w.b) * p.Hq + T.hq) * p.Nq + r] =
+          p.lse[VARLEN ? size_t(T.hq) * p.total_q + w.q0 + r : (size_t(w.b) * p.Hq + T.hq) * p.Nq + r] =
               (l > 0.f) ? fmaf(m, p.scale, __log2f(l) * 0.6931471805599453f) : -CUDART_INF_F;
       }
     }
@@ -497,10 +630,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       int kv = 0, qi = 0;                   // K/V ring position, items with a Q load
       bool alive = true;
       for (int k = 0; alive; ++k) {
-        const int item = item_of(p, k);
+        const int item = item_of(n_items, k);
         if (item < 0) break;
         WorkItem w;
-        decode_item(p, item, w);
+        decode_item<VARLEN>(p, item, w, vs);
         if (w.U == 0) continue;
         if (!(alive = wwait(L::B_Q, uint32_t(qi & 1)))) break;
         tc_fence_after();
@@ -556,10 +689,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       int issued_k = 0, issued_v = 0;
       bool alive = true;
       for (int k = 0; alive; ++k) {
-        const int item = item_of(p, k);
+        const int item = item_of(n_items, k);
         if (item < 0) break;
         WorkItem w;
-        decode_item(p, item, w);
+        decode_item<VARLEN>(p, item, w, vs);
         if (w.U == 0) continue;
         // Q buffers are free once every Q.K^T of the previous item completed
         if (qi > 0 && !(alive = mbar_wait(bar(L::B_QE), uint32_t((qi - 1) & 1), abort_flag))) break;
@@ -568,7 +701,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         for (int t = 0; t < 2; ++t)
           for (int c = 0; c < D / 64; ++c)
             tma_load_4d(sb + L::OFF_Q + t * L::TILE + c * L::HALF, &tmQ, bar(L::B_Q), c * 64,
-                        w.tile[t].hq, w.tile[t].row0, w.b);
+                        w.tile[t].hq, w.q0 + w.tile[t].row0, w.bc);
         ++qi;
         for (int it = 0; it < w.U; ++it, ++kv) {
           const int j = w.ubhi - 1 - it;
@@ -578,13 +711,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           mbar_arrive_expect_tx(bar(L::B_KF + slot), L::TILE);
           for (int c = 0; c < D / 64; ++c)
             tma_load_4d(sb + L::OFF_K + slot * L::TILE + c * L::HALF, &tmK, bar(L::B_KF + slot),
-                        c * 64, w.hkv, j * 128, w.b);
+                        c * 64, w.hkv, w.k0 + j * 128, w.bc);
           issued_k = kv + 1;
           if (!(alive = mbar_wait(bar(L::B_VE + slot), ph ^ 1u, abort_flag))) break;
           mbar_arrive_expect_tx(bar(L::B_VF + slot), L::TILE);
           for (int c = 0; c < D / 64; ++c)
             tma_load_4d(sb + L::OFF_V + slot * L::TILE + c * L::HALF, &tmV, bar(L::B_VF + slot),
-                        c * 64, w.hkv, j * 128, w.b);
+                        c * 64, w.hkv, w.k0 + j * 128, w.bc);
           issued_v = kv + 1;
         }
       }

@@ -13,6 +13,7 @@ namespace attn {
 __device__ int g_attn_status;
 
 constexpr int kStatusTimeout = 4;                     // == ATTN_ERR_TIMEOUT
+constexpr int kStatusBadInput = 1;                    // == ATTN_ERR_INVALID_ARG (device-side check)
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;   // 1 s per wait
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

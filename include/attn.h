@@ -53,7 +53,8 @@ extern "C" {
 
 typedef enum {
   ATTN_OK = 0,
-  ATTN_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misalignment, Hq % Hkv != 0, ... */
+  ATTN_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misalignment, Hq % Hkv != 0, ...;
+                                 also from attn_device_status after a device-side input check */
   ATTN_ERR_UNSUPPORTED = 2,   /* device is not sm_100, or head dim not in {64, 128} */
   ATTN_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed (message has the code) */
   ATTN_ERR_TIMEOUT = 4,       /* a bounded device-side wait gave up (see attn_device_status) */
@@ -79,6 +80,35 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
 int attn_fwd_f32o(const void* q, const void* k, const void* v, float* o, float* lse,
                   int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
                   int causal, int window_left, cudaStream_t stream);
+
+/*
+ * Forward pass over packed variable-length sequences (no padding): sequence b
+ * owns query rows [cu_seqlens_q[b], cu_seqlens_q[b+1]) of Q/O and keys
+ * [cu_seqlens_k[b], cu_seqlens_k[b+1]) of K/V, and attends only to its own
+ * keys with the mask convention above applied per sequence (qpos(i) =
+ * i + Nk_b - Nq_b). Packing sequences removes the work spent on padding, and
+ * packed sequence boundaries need variable-length kernels ("How to Reduce
+ * Attention Computation Cost in LLM Training": its FlashAttention section, its
+ * comparison table, and "How much does sequence packing actually help?").
+ * Each sequence's result is that of attn_fwd on it alone, bit for bit.
+ *   q   : device, bf16 [total_q, Hq, d];  k, v : device, bf16 [total_k, Hkv, d]
+ *   o   : device, bf16 [total_q, Hq, d] (rows of sequences are written; rows
+ *         outside every [cu_q[b], cu_q[b+1]) are left untouched)
+ *   lse : device, f32 [Hq, total_q], or NULL
+ *   cu_seqlens_q, cu_seqlens_k : device, int32 [B + 1], non-decreasing,
+ *         cu[0] >= 0, cu[B] <= total; 4-byte aligned
+ *   max_seqlen_q / max_seqlen_k : >= every sequence's length (host values;
+ *         they size the work list) and <= total_q / total_k
+ *   other arguments : as attn_fwd (B = number of sequences)
+ * The offsets are device data and are checked on the device: a sequence whose
+ * offsets fall outside the packed tensors or exceed the max lengths is
+ * skipped (nothing of it is written) and attn_device_status then returns
+ * ATTN_ERR_INVALID_ARG.
+ */
+int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                    const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int Hq, int Hkv,
+                    int total_q, int total_k, int max_seqlen_q, int max_seqlen_k, int d,
+                    float scale, int causal, int window_left, cudaStream_t stream);
 
 /*
  * Bytes of device workspace attn_decode needs for these sizes.

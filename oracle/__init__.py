@@ -13,6 +13,7 @@ from .attention import (  # noqa: F401
     allowed_mask,
     oracle_attention,
     oracle_attention_rows,
+    oracle_attention_varlen,
     oracle_decode,
     oracle_decode_paged,
     oracle_probabilities,

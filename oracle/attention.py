@@ -191,6 +191,39 @@ def oracle_decode(q, k_cache, v_cache, seqlens=None, window_left: int = -1,
     return O, LSE
 
 
+def oracle_attention_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, causal: bool = False,
+                            window_left: int = -1, scale: float | None = None):
+    """Attention over packed variable-length sequences.
+
+    Sequence ``b`` owns query rows ``[cu_q[b], cu_q[b+1])`` of ``q [total_q,
+    Hq, d]`` and keys ``[cu_k[b], cu_k[b+1])`` of ``k, v [total_k, Hkv, d]``
+    and attends to its own keys only, with the mask of ``allowed_mask`` taken
+    per sequence ("How to Reduce Attention Computation Cost in LLM Training":
+    packed sequence boundaries need variable-length kernels). Returns ``(O
+    [total_q, Hq, d], LSE [Hq, total_q])``; rows outside every sequence are
+    NaN (not computed).
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    cq = [int(x) for x in np.asarray(cu_seqlens_q).reshape(-1)]
+    ck = [int(x) for x in np.asarray(cu_seqlens_k).reshape(-1)]
+    total_q, Hq, d = q.shape
+    O = np.full((total_q, Hq, d), np.nan)
+    LSE = np.full((Hq, total_q), np.nan)
+    for b in range(len(cq) - 1):
+        q0, q1, k0, k1 = cq[b], cq[b + 1], ck[b], ck[b + 1]
+        if q1 <= q0:
+            continue
+        if k1 <= k0:                       # no keys: every row has no allowed key
+            O[q0:q1] = 0.0
+            LSE[:, q0:q1] = NEG_INF
+            continue
+        o, lse = oracle_attention(q[None, q0:q1], k[None, k0:k1], v[None, k0:k1], causal=causal,
+                                  window_left=window_left, scale=scale)
+        O[q0:q1] = o[0]
+        LSE[:, q0:q1] = lse[0]
+    return O, LSE
+
+
 def paged_to_contiguous(pages, block_table, seqlens=None):
     """Logical per-sequence cache from a paged pool.
 

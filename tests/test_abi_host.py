@@ -32,7 +32,8 @@ def header_functions():
 
 def test_header_declares_the_expected_entry_points():
     assert header_functions() == sorted([
-        "attn_fwd", "attn_fwd_f32o", "attn_decode_workspace_bytes", "attn_decode",
+        "attn_fwd", "attn_fwd_f32o", "attn_fwd_varlen", "attn_decode_workspace_bytes",
+        "attn_decode",
         "attn_decode_paged", "attn_decode_noalloc", "attn_last_error", "attn_device_status",
         "attn_launch_count",
         "attn_selftest_wait_timeout"])
@@ -117,6 +118,40 @@ def test_decode_rejects_bad_arguments_without_launch(lib, over, code):
     before = lib.attn_launch_count()
     rc = lib.attn_decode(*dec_args(**over))
     assert rc == code, lib.attn_last_error()
+    assert lib.attn_launch_count() == before
+
+
+def varlen_args(**over):
+    a = dict(q=P, k=P, v=P, o=P, lse=None, cq=P, ck=P, B=3, Hq=8, Hkv=2, total_q=900,
+             total_k=900, max_q=512, max_k=512, d=128, scale=0.1, causal=1, window_left=-1,
+             stream=None)
+    a.update(over)
+    return [a[k] for k in ("q", "k", "v", "o", "lse", "cq", "ck", "B", "Hq", "Hkv", "total_q",
+                           "total_k", "max_q", "max_k", "d", "scale", "causal", "window_left",
+                           "stream")]
+
+
+BAD_VARLEN = [
+    (dict(cq=None), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(ck=P + 2), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(total_q=0), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(max_q=1000), _lib.ATTN_ERR_INVALID_ARG),        # longer than total_q
+    (dict(max_k=0), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(B=0), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(Hq=6, Hkv=4), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(d=48), _lib.ATTN_ERR_UNSUPPORTED),
+    (dict(causal=2), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(o=P + 8), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(total_q=1 << 28, max_q=512, Hq=16, Hkv=2), _lib.ATTN_ERR_INVALID_ARG),
+]
+
+
+@pytest.mark.parametrize("over,code", BAD_VARLEN)
+def test_varlen_rejects_bad_arguments_without_launch(lib, over, code):
+    before = lib.attn_launch_count()
+    rc = lib.attn_fwd_varlen(*varlen_args(**over))
+    assert rc == code, lib.attn_last_error()
+    assert lib.attn_last_error()
     assert lib.attn_launch_count() == before
 
 
