@@ -515,7 +515,8 @@ def run_ours(args, world, rank, local):
             "roofline": {"bound": "tensor", "achieved": v_achieved, "peak": peak_t,
                          "unit": "TFLOP/s", "frac": v_achieved / peak_t,
                          "peak_source": f"{peak_src} bf16_tflops (burst)",
-                         "kernel": "attn_fwd_kernel<128,false> (packed)", "traffic": None},
+                         "kernel": "attn_fwd_kernel<128,false> (packed)",
+                         "traffic": recorded_traffic("attn_fwd_kernel", "varlen")},
             "gpu_launches": vlaunches,
         },
         "decode_paged": {
