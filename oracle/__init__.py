@@ -12,6 +12,7 @@ S and the probability matrix P exactly as the plain definition states
 from .attention import (  # noqa: F401
     allowed_mask,
     oracle_attention,
+    oracle_attention_backward,
     oracle_attention_rows,
     oracle_attention_varlen,
     oracle_decode,

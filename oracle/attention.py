@@ -191,6 +191,43 @@ def oracle_decode(q, k_cache, v_cache, seqlens=None, window_left: int = -1,
     return O, LSE
 
 
+def oracle_attention_backward(q, k, v, dout, causal: bool = False, window_left: int = -1,
+                              scale: float | None = None):
+    """Gradients of the plain definition: ``(dQ [B,Nq,Hq,d], dK, dV [B,Nk,Hkv,d])``.
+
+    The pages state the forward only and note that the saved log-sum-exp is
+    what a backward pass reuses ("Chapter 3 ...", section 3.5); the gradients
+    here are the exact derivatives of O = P V with P = softmax(scale Q Kᵀ +
+    mask), taken step by step:
+      dV = Pᵀ dO;  dP = dO Vᵀ;  dS = P * (dP - rowsum(P * dP));
+      dQ = scale dS K;  dK = scale dSᵀ Q.
+    rowsum(P * dP) equals rowsum(dO * O). With grouped heads a K/V head's
+    gradients sum those of its query heads. Rows with no allowed key
+    contribute nothing.
+    """
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, Nq, Hq, d = q.shape
+    _, Nk, Hkv, _ = k.shape
+    group = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    mask = allowed_mask(Nq, Nk, causal, window_left)
+    dQ = np.zeros_like(q)
+    dK = np.zeros_like(k)
+    dV = np.zeros_like(v)
+    for b in range(B):
+        for hq in range(Hq):
+            hk = hq // group
+            _, _, P = _head_attention(q[b, :, hq], k[b, :, hk], v[b, :, hk], scale, mask)
+            dO = do[b, :, hq]
+            dV[b, :, hk] += P.T @ dO
+            dP = dO @ v[b, :, hk].T
+            dS = P * (dP - (P * dP).sum(axis=1, keepdims=True))
+            dQ[b, :, hq] = scale * (dS @ k[b, :, hk])
+            dK[b, :, hk] += scale * (dS.T @ q[b, :, hq])
+    return dQ, dK, dV
+
+
 def oracle_attention_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, causal: bool = False,
                             window_left: int = -1, scale: float | None = None):
     """Attention over packed variable-length sequences.
