@@ -77,6 +77,11 @@ def make_decode(B, Hq, Hkv, Lmax, d, seed: int = SEED_Q):
     return q, k, v
 
 
+def make_dout(B, Nq, Hq, d, seed: int = SEED_Q + 21):
+    """bf16 CPU upstream gradient ``dO [B, Nq, Hq, d]`` (iid normal)."""
+    return _randn((B, Nq, Hq, d), seed)
+
+
 def make_for(w: Workload, seed: int = SEED_Q):
     if w.decode:
         return make_decode(w.B, w.Hq, w.Hkv, w.Nk, w.d, seed)

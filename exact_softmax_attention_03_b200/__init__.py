@@ -19,7 +19,8 @@ import torch
 
 from ._lib import AttnError, check, load  # noqa: F401
 
-__all__ = ["attn_fwd", "attn_fwd_f32o", "attn_fwd_varlen", "attn_decode", "attn_decode_paged",
+__all__ = ["attn_fwd", "attn_fwd_f32o", "attn_fwd_varlen", "attn_bwd", "attn_bwd_workspace_bytes",
+           "attn_decode", "attn_decode_paged",
            "attn_decode_workspace_bytes", "attn_decode_noalloc",
            "attn_device_status", "attn_last_error", "attn_launch_count", "AttnError"]
 
@@ -118,6 +119,43 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqle
                                  float(scale), int(bool(causal)), int(window_left),
                                  _stream_handle(stream)))
     return o, lse
+
+
+def attn_bwd_workspace_bytes(B: int, Hq: int, Nq: int, d: int) -> int:
+    return int(load().attn_bwd_workspace_bytes(B, Hq, Nq, d))
+
+
+def attn_bwd(q, k, v, o, lse, dout, causal=False, window_left=-1, scale=None, dq=None, dk=None,
+             dv=None, workspace=None, stream=None):
+    """Gradients of :func:`attn_fwd`. Returns ``(dq, dk, dv)`` (bf16).
+
+    ``o`` and ``lse`` are what ``attn_fwd`` returned for the same inputs and
+    mask; ``dout`` is the upstream gradient, shaped like ``o``. ``workspace``
+    (``attn_bwd_workspace_bytes(...)`` bytes) is allocated here if not given.
+    """
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        _need(t, n, torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32, 3)
+    B, Nq, Hq, d = q.shape
+    _, Nk, Hkv, _ = k.shape
+    if o.shape != q.shape or dout.shape != q.shape or v.shape != k.shape:
+        raise ValueError("o and dout must be shaped like q, v like k")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _need(t, n, torch.bfloat16, 4)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    need = attn_bwd_workspace_bytes(B, Hq, Nq, d)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    check(load().attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
+                          lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv,
+                          Nq, Nk, d, float(scale), int(bool(causal)), int(window_left),
+                          workspace.data_ptr(), ws_bytes, _stream_handle(stream)))
+    return dq, dk, dv
 
 
 def attn_decode_workspace_bytes(B: int, Hq: int, d: int, num_splits: int = 0, Lmax: int = 1) -> int:

@@ -14,6 +14,7 @@
 #include <mutex>
 
 #include "../../include/attn.h"
+#include "backward_kernels.cuh"
 #include "decode_kernels.cuh"
 #include "prefill_kernel.cuh"
 
@@ -350,6 +351,43 @@ int noalloc_scratch(int dev, void** out) {
   return ATTN_OK;
 }
 
+// ---------------------------------------------------------------- backward --
+
+size_t bwd_ws_dq_bytes(int B, int Hq, int Nq, int d) {
+  return (static_cast<size_t>(B) * Nq * Hq * d * sizeof(float) + 255) / 256 * 256;
+}
+size_t bwd_ws_bytes(int B, int Hq, int Nq, int d) {
+  return bwd_ws_dq_bytes(B, Hq, Nq, d) +
+         (static_cast<size_t>(B) * Hq * Nq * sizeof(float) + 255) / 256 * 256;
+}
+
+template <int D>
+int launch_bwd(const void* q, const void* k, const void* v, attn::BwdParams& p, cudaStream_t stream,
+               int dev) {
+  using L = attn::BwdLayout<D>;
+  CUtensorMap mq, mk, mv, mdo;
+  int rc;
+  if ((rc = make_map(&mq, q, D, p.Hq, p.Nq, p.B)) != ATTN_OK) return rc;
+  if ((rc = make_map(&mk, k, D, p.Hkv, p.Nk, p.B)) != ATTN_OK) return rc;
+  if ((rc = make_map(&mv, v, D, p.Hkv, p.Nk, p.B)) != ATTN_OK) return rc;
+  if ((rc = make_map(&mdo, p.dout, D, p.Hq, p.Nq, p.B)) != ATTN_OK) return rc;
+  static std::atomic<unsigned long long> attr_set{0};   // per-device bit
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(attr_set.load() & bit)) {
+    cudaError_t e = cudaFuncSetAttribute(attn::bwd_main_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_ALLOC);
+    if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    attr_set.fetch_or(bit);
+  }
+  const long long rows = static_cast<long long>(p.B) * p.Nq * p.Hq;
+  attn::bwd_prep_kernel<D><<<unsigned((rows * 32 + 255) / 256), 256, 0, stream>>>(p);
+  const dim3 grid(unsigned((p.Nk + 127) / 128), unsigned(p.Hkv), unsigned(p.B));
+  attn::bwd_main_kernel<D><<<grid, attn::kBwdThreads, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, p);
+  const long long n8 = rows * D / 8;
+  attn::bwd_finalize_kernel<<<unsigned((n8 + 255) / 256), 256, 0, stream>>>(p, n8);
+  return ATTN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -435,6 +473,52 @@ int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float*
   const Packed pk{cu_seqlens_q, cu_seqlens_k, total_q, total_k};
   return fwd_entry(q, k, v, o, lse, B, Hq, Hkv, max_seqlen_q, max_seqlen_k, d, scale, causal,
                    window_left, stream, false, &pk);
+}
+
+size_t attn_bwd_workspace_bytes(int B, int Hq, int Nq, int d) {
+  if (B < 1 || Hq < 1 || Nq < 1 || (d != 64 && d != 128)) return 0;
+  return bwd_ws_bytes(B, Hq, Nq, d);
+}
+
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+             const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nk,
+             int d, float scale, int causal, int window_left, void* workspace,
+             size_t workspace_bytes, cudaStream_t stream) {
+  int rc = validate_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal);
+  if (rc != ATTN_OK) return rc;
+  if (!dout || !lse || !dq || !dk || !dv)
+    return fail(ATTN_ERR_INVALID_ARG, "dout, lse, dq, dk and dv must be non-null");
+  if (!aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16))
+    return fail(ATTN_ERR_INVALID_ARG, "dout, dq, dk, dv must be 16-byte aligned");
+  if (static_cast<long long>(B) * Nq * Hq * d > kMaxIndex * 8ll)
+    return fail(ATTN_ERR_INVALID_ARG, "sizes too large");
+  const size_t need = bwd_ws_bytes(B, Hq, Nq, d);
+  if (workspace == nullptr || workspace_bytes < need)
+    return fail(ATTN_ERR_WORKSPACE, "workspace of %zu bytes needed, got %zu", need,
+                workspace == nullptr ? size_t(0) : workspace_bytes);
+  if (!aligned(workspace, 256)) return fail(ATTN_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  int dev = 0;
+  if ((rc = check_device(&dev)) != ATTN_OK) return rc;
+  attn::BwdParams p{};
+  p.o = static_cast<const uint16_t*>(o);
+  p.dout = static_cast<const uint16_t*>(dout);
+  p.lse = lse;
+  p.dq_acc = static_cast<float*>(workspace);
+  p.delta = reinterpret_cast<float*>(static_cast<char*>(workspace) + bwd_ws_dq_bytes(B, Hq, Nq, d));
+  p.dq = static_cast<uint16_t*>(dq);
+  p.dk = static_cast<uint16_t*>(dk);
+  p.dv = static_cast<uint16_t*>(dv);
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Nq = Nq; p.Nk = Nk;
+  p.causal = causal;
+  p.window_left = window_left < 0 ? -1 : window_left;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  rc = d == 128 ? launch_bwd<128>(q, k, v, p, stream, dev) : launch_bwd<64>(q, k, v, p, stream, dev);
+  if (rc != ATTN_OK) return rc;
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "attn_bwd launch: %s", cudaGetErrorString(e));
+  g_launches.fetch_add(3);
+  return ok();
 }
 
 size_t attn_decode_workspace_bytes(int B, int Hq, int d, int num_splits, int Lmax) {

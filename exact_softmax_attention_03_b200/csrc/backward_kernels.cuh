@@ -1,0 +1,440 @@
+// backward_kernels.cuh — gradients of exact attention on sm_100a tensor cores.
+//
+// For O = P V with P = softmax(scale * Q Kᵀ + mask), the gradients are
+//   dV = Pᵀ dO,  dP = dO Vᵀ,  dS = P * (dP - rowsum(dO * O)),
+//   dQ = scale * dS K,  dK = scale * dSᵀ Q,
+// with P recomputed from the log-sum-exp the forward pass saved ("Chapter 3:
+// MHA Limitations, MQA, GQA, and FlashAttention", section 3.5: the saved
+// log-sum-exp serves the backward pass), so no score matrix is stored.
+//
+// Three kernels:
+//   bwd_prep_kernel     delta = rowsum(dO * O) per query row; zeroes the fp32
+//                       dQ accumulator
+//   bwd_main_kernel     one CTA per (batch, K/V head, 128-key block): loops
+//                       over the group's query heads and the query blocks the
+//                       mask allows, accumulates dK and dV of its keys in
+//                       tensor memory, adds dQ contributions to the
+//                       accumulator with vector atomics
+//   bwd_finalize_kernel dQ accumulator -> bf16
+//
+// bwd_main_kernel warp roles (192 threads):
+//   warps 0-3  elementwise, thread = TMEM lane: first a key row (P, dS), then
+//              a query row (reading dQ); at the end a key row again (dK, dV)
+//   warp 4     tensor-core issuer (whole warp, one elected lane issues)
+//   warp 5     TMA producer (one lane): K_j, V_j once; Q_i, dO_i per block
+// Per query block (tile = 128 x 128):
+//   Sᵀ  = K_j Q_iᵀ        SS, both K-major                 -> TMEM cols [0,128)
+//   dPᵀ = V_j dO_iᵀ       SS, both K-major                 -> TMEM cols [128,256)
+//   elementwise: Pᵀ = exp2(Sᵀ c - lse2), dSᵀ = Pᵀ (dPᵀ - delta); Pᵀ and dSᵀ
+//     as bf16 pairs over cols [0,64) and [128,192); dSᵀ also to shared memory
+//   dV += Pᵀ dO_i         TS: A = Pᵀ (TMEM), B = dO_i MN-major
+//   dK += dSᵀ Q_i         TS: A = dSᵀ (TMEM), B = Q_i MN-major
+//   dQ_i = dS K_j         SS: A = dS MN-major (the dSᵀ tile read transposed),
+//                         B = K_j MN-major; 64 columns of d at a time into the
+//                         free cols [64,128) and [192,256)
+// All waits are bounded (sm100_ptx.cuh).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include "sm100_ptx.cuh"
+
+namespace attn {
+
+// kind::f16 instruction descriptor with A MN-major too (bit 15).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_amn(int M, int N, int b_mn_major) {
+  return idesc_bf16_f32(M, N, b_mn_major) | (1u << 15);
+}
+
+struct BwdParams {
+  const uint16_t* o;       // [B, Nq, Hq, D] bf16, forward output
+  const uint16_t* dout;    // [B, Nq, Hq, D] bf16
+  const float* lse;        // [B, Hq, Nq] natural log-sum-exp of the forward
+  float* delta;            // [B, Hq, Nq] rowsum(dO * O)              (workspace)
+  float* dq_acc;           // [B, Nq, Hq, D] fp32, scale * dQ         (workspace)
+  uint16_t* dq;            // [B, Nq, Hq, D] bf16
+  uint16_t* dk;            // [B, Nk, Hkv, D] bf16
+  uint16_t* dv;            // [B, Nk, Hkv, D] bf16
+  int B, Hq, Hkv, Nq, Nk;
+  int causal, window_left;
+  float scale, scale_log2;
+};
+
+// ---- delta = rowsum(dO * O); zero the dQ accumulator ------------------------
+// One warp per (b, query row, head); lane l covers elements [l*D/32, (l+1)*D/32).
+template <int D>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p) {
+  constexpr int EPL = D / 32;
+  const long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long rows = static_cast<long long>(p.B) * p.Nq * p.Hq;
+  if (row >= rows) return;
+  const size_t base = size_t(row) * D + lane * EPL;          // row = (b * Nq + q) * Hq + h
+  float acc = 0.f;
+#pragma unroll
+  for (int e = 0; e < EPL; e += 2) {
+    const uint32_t a = *reinterpret_cast<const uint32_t*>(p.dout + base + e);
+    const uint32_t c = *reinterpret_cast<const uint32_t*>(p.o + base + e);
+    acc = fmaf(bf16lo(a), bf16lo(c), acc);
+    acc = fmaf(bf16hi(a), bf16hi(c), acc);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) p.dq_acc[base + e] = 0.f;
+  if (lane == 0) {
+    const int h = int(row % p.Hq);
+    const long long bq = row / p.Hq;                         // b * Nq + q
+    const int q = int(bq % p.Nq);
+    const int b = int(bq / p.Nq);
+    p.delta[(size_t(b) * p.Hq + h) * p.Nq + q] = acc;
+  }
+}
+
+// ---- dQ accumulator (already scaled) -> bf16 --------------------------------
+__global__ void __launch_bounds__(256) bwd_finalize_kernel(const BwdParams p, long long n8) {
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const float4 a = reinterpret_cast<const float4*>(p.dq_acc)[2 * i];
+  const float4 b = reinterpret_cast<const float4*>(p.dq_acc)[2 * i + 1];
+  uint4 v;
+  v.x = pack_bf16x2(a.x, a.y);
+  v.y = pack_bf16x2(a.z, a.w);
+  v.z = pack_bf16x2(b.x, b.y);
+  v.w = pack_bf16x2(b.z, b.w);
+  reinterpret_cast<uint4*>(p.dq)[i] = v;
+}
+
+template <int D>
+struct BwdLayout {
+  static constexpr int TILE = 128 * D * 2;                 // 128 rows x D bf16
+  static constexpr int HALF = 128 * 128;                   // 128 rows x 64 columns, swizzled
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + TILE;
+  static constexpr int OFF_Q = OFF_V + TILE;
+  static constexpr int OFF_DO = OFF_Q + TILE;
+  static constexpr int OFF_DS = OFF_DO + TILE;             // dSᵀ [128 keys][128 queries] bf16
+  static constexpr int OFF_LD = OFF_DS + 2 * HALF;         // f32 lse2[2][128], delta[2][128]
+  static constexpr int OFF_BAR = OFF_LD + 4 * 128 * 4;
+  static constexpr int B_KV = 0;     // K_j, V_j loaded
+  static constexpr int B_QD = 1;     // Q_i, dO_i loaded
+  static constexpr int B_QDE = 2;    // Q_i, dO_i and the dS tile free again
+  static constexpr int B_SD = 3;     // Sᵀ and dPᵀ in TMEM
+  static constexpr int B_PR = 4;     // Pᵀ, dSᵀ written (128 arrivals)
+  static constexpr int B_QR = 5;     // dQ_i in TMEM
+  static constexpr int B_QF = 6;     // dQ_i read (128 arrivals)
+  static constexpr int B_DONE = 7;   // every dK / dV product complete
+  static constexpr int B_LD = 8;     // per-block lse2 / delta values in shared memory (128 arrivals)
+  static constexpr int NBAR = 9;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;      // [0] TMEM base, [1] abort flag
+  static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int SMEM_ALLOC = BYTES + 1024;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t COL_ST = 0, COL_DPT = 128, COL_DV = 256, COL_DK = 256 + D;
+  static constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, 0);
+  static constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, D, 1);
+  static constexpr uint32_t IDESC_DQ = idesc_bf16_f32_amn(128, 64, 1);
+};
+
+constexpr int kBwdThreads = 192;
+
+// Query blocks that hold at least one allowed (query, key) pair with a key in
+// [kb0, kb1]: [i_lo, i_hi], empty when i_hi < i_lo.
+__device__ __forceinline__ void bwd_qblocks(const BwdParams& p, int kb0, int kb1, int& i_lo, int& i_hi) {
+  const int off = p.Nk - p.Nq;                               // qpos = q + off
+  int q_lo = p.causal ? max(0, kb0 - off) : 0;
+  int q_hi = p.window_left >= 0 ? min(p.Nq - 1, kb1 + p.window_left - off) : p.Nq - 1;
+  if (q_hi < q_lo) { i_lo = 0; i_hi = -1; return; }
+  i_lo = q_lo / 128;
+  i_hi = q_hi / 128;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                const BwdParams p) {
+  using L = BwdLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  auto bar = [&](int i) -> uint32_t { return sb + L::OFF_BAR + 8u * uint32_t(i); };
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const int j = blockIdx.x, hkv = blockIdx.y, b = blockIdx.z;
+  const int G = p.Hq / p.Hkv;
+  const int kb0 = j * 128, kb1 = min(kb0 + 127, p.Nk - 1);
+  int i_lo, i_hi;
+  bwd_qblocks(p, kb0, kb1, i_lo, i_hi);
+  const int nblk = i_hi - i_lo + 1;                          // per query head (<= 0: none)
+  const int total = nblk > 0 ? G * nblk : 0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(L::B_KV), 1);
+    mbar_init(bar(L::B_QD), 1);
+    mbar_init(bar(L::B_QDE), 1);
+    mbar_init(bar(L::B_SD), 1);
+    mbar_init(bar(L::B_PR), 128);
+    mbar_init(bar(L::B_QR), 1);
+    mbar_init(bar(L::B_QF), 128);
+    mbar_init(bar(L::B_DONE), 1);
+    mbar_init(bar(L::B_LD), 128);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(smem_u32(tmem_holder), L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp < 4) {
+    // ======================= elementwise warps ==============================
+    const int t = int(threadIdx.x);                          // TMEM lane
+    const uint32_t lane_off = uint32_t(warp * 32) << 16;
+    const uint32_t tST = tmem + lane_off + L::COL_ST, tDPT = tmem + lane_off + L::COL_DPT;
+    float* lse2_s = reinterpret_cast<float*>(smem + L::OFF_LD);          // [2][128]
+    float* delta_s = lse2_s + 2 * 128;                                   // [2][128]
+    const int key = kb0 + t;
+    const int off = p.Nk - p.Nq;
+    const float c2 = p.scale_log2;
+    bool ok = true;
+    for (int n = 0; ok && n < total; ++n) {
+      const int g = n / nblk, i = i_lo + n % nblk;
+      const int hq = hkv * G + g;
+      const int par = n & 1;
+      {
+        const int q = i * 128 + t;
+        const bool qv = q < p.Nq;
+        const float l = qv ? __ldg(p.lse + (size_t(b) * p.Hq + hq) * p.Nq + q) : 0.f;
+        lse2_s[par * 128 + t] = (qv && l > -CUDART_INF_F) ? l * 1.4426950408889634f : 0.f;
+        delta_s[par * 128 + t] = qv ? __ldg(p.delta + (size_t(b) * p.Hq + hq) * p.Nq + q) : 0.f;
+      }
+      mbar_arrive(bar(L::B_LD));
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_LD), uint32_t(par), abort_flag)))) break;
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_SD), uint32_t(par), abort_flag)))) break;
+      tc_fence_after();
+      // allowed queries of this key within the block: [c_lo, c_hi]
+      const int q0 = i * 128;
+      int c_lo = 0, c_hi = min(127, p.Nq - 1 - q0);
+      if (key >= p.Nk) c_hi = -1;
+      if (p.causal) c_lo = max(c_lo, key - off - q0);                    // key <= q + off
+      if (p.window_left >= 0) c_hi = min(c_hi, key + p.window_left - off - q0);
+      const float* lsr = lse2_s + par * 128;
+      const float* dlt = delta_s + par * 128;
+      // 64 queries at a time: read their Sᵀ and dPᵀ columns (32 at a time),
+      // then write the bf16 pairs of Pᵀ and dSᵀ over columns already read
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pw[32], dw[32];
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c0 = 64 * h + 32 * cc;
+          uint32_t sr[32], dr[32];
+          tmem_ld32(tST + c0, sr);
+          tmem_ld32(tDPT + c0, dr);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            float pp[2], ds[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int c = c0 + e + u;
+              const bool al = c >= c_lo && c <= c_hi;
+              const float x = fmaf(__uint_as_float(sr[e + u]), c2, -lsr[c]);
+              pp[u] = al ? ex2_approx(x) : 0.f;
+              ds[u] = pp[u] * (__uint_as_float(dr[e + u]) - dlt[c]);
+            }
+            pw[16 * cc + e / 2] = pack_bf16x2(pp[0], pp[1]);
+            dw[16 * cc + e / 2] = pack_bf16x2(ds[0], ds[1]);
+          }
+        }
+        tmem_st32(tST + 32 * h, pw);
+        tmem_st32(tDPT + 32 * h, dw);
+        // dSᵀ row of this key -> shared memory block h (queries 64h..64h+63),
+        // 16-byte chunks swizzled by (row & 7)
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint32_t addr = sb + L::OFF_DS + h * L::HALF + t * 128 + ((ch ^ (t & 7)) * 16);
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
+                       ::"r"(addr), "r"(dw[4 * ch]), "r"(dw[4 * ch + 1]), "r"(dw[4 * ch + 2]),
+                       "r"(dw[4 * ch + 3]) : "memory");
+        }
+      }
+      tmem_wait_st();
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      tc_fence_before();
+      mbar_arrive(bar(L::B_PR));
+      // ---- dQ rows: thread t is now query row q0 + t ----------------------
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_QR), uint32_t(par), abort_flag)))) break;
+      tc_fence_after();
+      uint32_t qr[D];
+#pragma unroll
+      for (int h = 0; h < D / 64; ++h) {
+        const uint32_t col = (h == 0 ? tST : tDPT) + 64;
+        tmem_ld32(col, qr + 64 * h);
+        tmem_ld32(col + 32, qr + 64 * h + 32);
+      }
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar(L::B_QF));
+      const int q = q0 + t;
+      if (q < p.Nq) {
+        float4* dst = reinterpret_cast<float4*>(p.dq_acc + ((size_t(b) * p.Nq + q) * p.Hq + hq) * D);
+#pragma unroll
+        for (int e = 0; e < D / 4; ++e)
+          atomicAdd(dst + e, make_float4(__uint_as_float(qr[4 * e]) * p.scale,
+                                         __uint_as_float(qr[4 * e + 1]) * p.scale,
+                                         __uint_as_float(qr[4 * e + 2]) * p.scale,
+                                         __uint_as_float(qr[4 * e + 3]) * p.scale));
+      }
+    }
+    // ---- dK, dV of this key row ---------------------------------------------
+    const bool have = ok && total > 0 &&
+                      __all_sync(0xffffffffu, mbar_wait(bar(L::B_DONE), 0u, abort_flag));
+    if (have) tc_fence_after();
+    // tcgen05.ld is warp-collective: every lane loads; only the stores of
+    // keys inside the sequence are guarded
+    if (have || (ok && total == 0)) {
+      const size_t base = ((size_t(b) * p.Nk + min(key, p.Nk - 1)) * p.Hkv + hkv) * D;
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {                          // 0: dV, 1: dK (scaled)
+        uint4* dst = reinterpret_cast<uint4*>((m ? p.dk : p.dv) + base);
+        const float f = m ? p.scale : 1.f;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          if (have) {
+            __syncwarp();
+            tmem_ld32(tmem + lane_off + (m ? L::COL_DK : L::COL_DV) + 32 * c, r);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = 0u;
+          }
+          if (key >= p.Nk) continue;
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[4 * c + e] = make_uint4(
+                pack_bf16x2(__uint_as_float(r[8 * e]) * f, __uint_as_float(r[8 * e + 1]) * f),
+                pack_bf16x2(__uint_as_float(r[8 * e + 2]) * f, __uint_as_float(r[8 * e + 3]) * f),
+                pack_bf16x2(__uint_as_float(r[8 * e + 4]) * f, __uint_as_float(r[8 * e + 5]) * f),
+                pack_bf16x2(__uint_as_float(r[8 * e + 6]) * f, __uint_as_float(r[8 * e + 7]) * f));
+        }
+      }
+    }
+  } else if (warp == 4) {
+    // ======================= tensor-core issuer ==============================
+    auto wwait = [&](int bi, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar(bi), parity, abort_flag));
+    };
+    auto commit = [&](int bi) { if (elect_one()) tc_commit(bar(bi)); };
+    // K-major views (Sᵀ, dPᵀ) and MN-major views (dK, dV, dQ) of the same tiles
+    const uint64_t dK_k = smem_desc_sw128(sb + L::OFF_K, 16, 1024);
+    const uint64_t dV_k = smem_desc_sw128(sb + L::OFF_V, 16, 1024);
+    const uint64_t dQ_k = smem_desc_sw128(sb + L::OFF_Q, 16, 1024);
+    const uint64_t dO_k = smem_desc_sw128(sb + L::OFF_DO, 16, 1024);
+    const uint64_t dQ_mn = smem_desc_sw128(sb + L::OFF_Q, L::HALF, 1024);
+    const uint64_t dO_mn = smem_desc_sw128(sb + L::OFF_DO, L::HALF, 1024);
+    const uint64_t dS_mn = smem_desc_sw128(sb + L::OFF_DS, L::HALF, 1024);
+    const uint64_t dKj_mn = smem_desc_sw128(sb + L::OFF_K, L::HALF, 1024);
+    const uint32_t tST = tmem + L::COL_ST, tDPT = tmem + L::COL_DPT;
+    const uint32_t tDV = tmem + L::COL_DV, tDK = tmem + L::COL_DK;
+    bool alive = total > 0 && wwait(L::B_KV, 0u);
+    for (int n = 0; alive && n < total; ++n) {
+      const uint32_t par = uint32_t(n & 1);
+      if (!(alive = wwait(L::B_QD, par))) break;
+      if (n > 0 && !(alive = wwait(L::B_QF, par ^ 1u))) break;   // previous dQ read out
+      tc_fence_after();
+      // Sᵀ = K_j Q_iᵀ and dPᵀ = V_j dO_iᵀ (K = d)
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t o = ((k / 4) * L::HALF + (k % 4) * 32) >> 4;
+        if (elect_one()) mma_ss(tST, dK_k + o, dQ_k + o, L::IDESC_S, k > 0 ? 1u : 0u);
+      }
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t o = ((k / 4) * L::HALF + (k % 4) * 32) >> 4;
+        if (elect_one()) mma_ss(tDPT, dV_k + o, dO_k + o, L::IDESC_S, k > 0 ? 1u : 0u);
+      }
+      commit(L::B_SD);
+      if (!(alive = wwait(L::B_PR, par))) break;
+      tc_fence_after();
+      // dV += Pᵀ dO_i, dK += dSᵀ Q_i (K = 128 queries, 16 per MMA)
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint32_t o = (k * 16 * 128) >> 4;
+        if (elect_one()) mma_ts(tDV, tST + 8 * k, dO_mn + o, L::IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint32_t o = (k * 16 * 128) >> 4;
+        if (elect_one()) mma_ts(tDK, tDPT + 8 * k, dQ_mn + o, L::IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
+      }
+      // dQ_i = dS K_j, 64 columns of d at a time (K = 128 keys)
+#pragma unroll
+      for (int h = 0; h < D / 64; ++h) {
+        const uint32_t dst = (h == 0 ? tST : tDPT) + 64;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t o = (k * 16 * 128) >> 4;
+          if (elect_one())
+            mma_ss(dst, dS_mn + o, dKj_mn + ((h * L::HALF) >> 4) + o, L::IDESC_DQ, k > 0 ? 1u : 0u);
+        }
+      }
+      commit(L::B_QR);
+      commit(L::B_QDE);
+    }
+    if (total > 0) {
+      commit(L::B_DONE);                        // also drains every issued product
+      mbar_wait(bar(L::B_DONE), 0, nullptr);
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    // ======================= TMA producer ====================================
+    if (lane == 0 && total > 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmDO);
+      mbar_arrive_expect_tx(bar(L::B_KV), 2 * L::TILE);
+      for (int c = 0; c < D / 64; ++c) {
+        tma_load_4d(sb + L::OFF_K + c * L::HALF, &tmK, bar(L::B_KV), c * 64, hkv, kb0, b);
+        tma_load_4d(sb + L::OFF_V + c * L::HALF, &tmV, bar(L::B_KV), c * 64, hkv, kb0, b);
+      }
+      int issued = 0;
+      for (int n = 0; n < total; ++n) {
+        const int g = n / nblk, i = i_lo + n % nblk;
+        const int hq = hkv * G + g;
+        if (n > 0 && !mbar_wait(bar(L::B_QDE), uint32_t((n - 1) & 1), abort_flag)) break;
+        mbar_arrive_expect_tx(bar(L::B_QD), 2 * L::TILE);
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_4d(sb + L::OFF_Q + c * L::HALF, &tmQ, bar(L::B_QD), c * 64, hq, i * 128, b);
+          tma_load_4d(sb + L::OFF_DO + c * L::HALF, &tmDO, bar(L::B_QD), c * 64, hq, i * 128, b);
+        }
+        issued = n + 1;
+      }
+      // no copy may still be landing at exit
+      mbar_wait(bar(L::B_KV), 0, nullptr);
+      if (issued > 0) mbar_wait(bar(L::B_QD), uint32_t((issued - 1) & 1), nullptr);
+    }
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::TMEM_COLS);
+  }
+}
+
+}  // namespace attn

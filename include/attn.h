@@ -111,6 +111,27 @@ int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float*
                     float scale, int causal, int window_left, cudaStream_t stream);
 
 /*
+ * Backward pass: gradients dQ, dK, dV of the attn_fwd operation for an
+ * upstream gradient dO, with P recomputed from the forward's LSE ("Chapter 3:
+ * MHA Limitations, MQA, GQA, and FlashAttention", section 3.5: the saved
+ * log-sum-exp serves the backward pass). dV = Pᵀ dO; dS = P * (dP - rowsum(dO
+ * * O)) with dP = dO Vᵀ; dQ = scale dS K; dK = scale dSᵀ Q; a K/V head's
+ * gradients sum over its group's query heads.
+ *   q, k, v, o, dout : device bf16, layouts of attn_fwd (o = its output)
+ *   lse  : device f32 [B, Hq, Nq], the LSE attn_fwd wrote for this o
+ *   dq   : device bf16 [B, Nq, Hq, d];  dk, dv : device bf16 [B, Nk, Hkv, d]
+ *   workspace : device, >= attn_bwd_workspace_bytes(B, Hq, Nq, d) bytes,
+ *          256-byte aligned (fp32 dQ accumulator and per-row dO.O sums)
+ *   other arguments : as attn_fwd (the same causal / window_left / scale)
+ * Returns ATTN_OK or an attn_status; nothing is launched on error.
+ */
+size_t attn_bwd_workspace_bytes(int B, int Hq, int Nq, int d);
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+             const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq,
+             int Nk, int d, float scale, int causal, int window_left, void* workspace,
+             size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * Bytes of device workspace attn_decode needs for these sizes.
  * num_splits = 0 picks the split count attn_decode would pick automatically.
  * Returns 0 for invalid sizes.
