@@ -376,6 +376,27 @@ def run_ours(args, world, rank, local):
     tiles = metrics.executed_tiles(w.Nq, w.Nk, w.causal, w.window_left) * w.B * w.Hq
     clocks = sampler.summary()
 
+    # backward leg on the same workload: dQ, dK, dV from the forward's O and LSE
+    # (2.5x the forward's mask-adjusted FLOPs: five products instead of two)
+    do_h = ai.make_dout(w.B, w.Nq, w.Hq, w.d, seed=shard_seed(rank) + 21)
+    dout = do_h.to(dev)
+    ea.attn_fwd(q, k, v, o=o, lse=lse, causal=w.causal, window_left=w.window_left)
+    dq_t, dk_t, dv_t = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    bws = torch.empty(ea.attn_bwd_workspace_bytes(w.B, w.Hq, w.Nq, w.d), dtype=torch.uint8,
+                      device=dev)
+
+    def bwd():
+        ea.attn_bwd(q, k, v, o, lse, dout, causal=w.causal, window_left=w.window_left,
+                    dq=dq_t, dk=dk_t, dv=dv_t, workspace=bws)
+
+    btimes, blaunches = timed_kernel_loop(bwd, args.steps, args.warmup, world, flush, None)
+    bms = statistics.mean(btimes)
+    bms_max = max_over_ranks(bms, world)
+    b_flops = 2.5 * flops
+    b_value = whole_job_rate(b_flops, bms_max, world) / 1e12
+    b_achieved = b_flops / (bms * 1e-3) / 1e12
+    del dout, dq_t, dk_t, dv_t, bws
+
     # packed variable-length prefill leg: 16 causal sequences with seeded
     # lengths in [256, 4096], MHA H32 d128, no padding
     vl_lens = ai.varlen_lengths(16, 256, 4096, seed=shard_seed(rank) + 13)
@@ -507,6 +528,17 @@ def run_ours(args, world, rank, local):
                          "algorithmic_bytes": d_all,
                          "traffic": recorded_traffic("decode", "decode")},
             "gpu_launches": dlaunches,
+        },
+        "backward": {
+            "workload": f"{w.name}, backward (dQ, dK, dV)", "value": b_value, "unit": "TFLOP/s",
+            "ms_per_step": bms_max,
+            "flop_count": "2.5 x the forward's mask-adjusted FLOPs",
+            "roofline": {"bound": "tensor", "achieved": b_achieved, "peak": peak_t,
+                         "unit": "TFLOP/s", "frac": b_achieved / peak_t,
+                         "peak_source": f"{peak_src} bf16_tflops (burst)",
+                         "kernel": "bwd_prep_kernel + bwd_main_kernel<128> + bwd_finalize_kernel",
+                         "traffic": None},
+            "gpu_launches": blaunches,
         },
         "varlen": {
             "workload": f"MHA causal packed prefill, 16 sequences of {min(vl_lens)}-{max(vl_lens)} "

@@ -122,6 +122,46 @@ def test_decode_rejects_bad_arguments_without_launch(lib, over, code):
     assert lib.attn_launch_count() == before
 
 
+def bwd_args(**over):
+    a = dict(q=P, k=P, v=P, o=P, do=P, lse=P, dq=P, dk=P, dv=P, B=2, Hq=8, Hkv=2, Nq=256, Nk=256,
+             d=128, scale=0.1, causal=1, window_left=-1, ws=P, ws_bytes=1 << 30, stream=None)
+    a.update(over)
+    return [a[k] for k in ("q", "k", "v", "o", "do", "lse", "dq", "dk", "dv", "B", "Hq", "Hkv",
+                           "Nq", "Nk", "d", "scale", "causal", "window_left", "ws", "ws_bytes",
+                           "stream")]
+
+
+BAD_BWD = [
+    (dict(do=None), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(lse=None), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(dk=None), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(dq=P + 8), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(Hq=6, Hkv=4), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(d=80), _lib.ATTN_ERR_UNSUPPORTED),
+    (dict(Nk=0), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(ws=None), _lib.ATTN_ERR_WORKSPACE),
+    (dict(ws_bytes=1000), _lib.ATTN_ERR_WORKSPACE),
+    (dict(ws=P + 16), _lib.ATTN_ERR_INVALID_ARG),
+]
+
+
+@pytest.mark.parametrize("over,code", BAD_BWD)
+def test_backward_rejects_bad_arguments_without_launch(lib, over, code):
+    before = lib.attn_launch_count()
+    rc = lib.attn_bwd(*bwd_args(**over))
+    assert rc == code, lib.attn_last_error()
+    assert lib.attn_last_error()
+    assert lib.attn_launch_count() == before
+
+
+def test_backward_workspace_bytes(lib):
+    f = lib.attn_bwd_workspace_bytes
+    assert f(0, 8, 128, 128) == 0 and f(1, 8, 128, 96) == 0
+    # fp32 dQ accumulator + per-row sums, each rounded to 256 bytes
+    assert f(2, 8, 100, 128) == ((2 * 100 * 8 * 128 * 4 + 255) // 256 * 256
+                                 + (2 * 8 * 100 * 4 + 255) // 256 * 256)
+
+
 def varlen_args(**over):
     a = dict(q=P, k=P, v=P, o=P, lse=None, cq=P, ck=P, B=3, Hq=8, Hkv=2, total_q=900,
              total_k=900, max_q=512, max_k=512, d=128, scale=0.1, causal=1, window_left=-1,
