@@ -397,6 +397,28 @@ def run_ours(args, world, rank, local):
     b_achieved = b_flops / (bms * 1e-3) / 1e12
     del dout, dq_t, dk_t, dv_t, bws
 
+    # merge leg (sequence-sharded attention's combine): 4 fp32 parts of the
+    # prefill output shape -> bf16 O and LSE; HBM-bound, inputs far above L2
+    R_m = 4
+    g_m = torch.Generator(device="cpu")
+    g_m.manual_seed(shard_seed(rank) + 31)
+    mo_parts = torch.randn((R_m, w.B, w.Nq, w.Hq, w.d), generator=g_m).to(dev)
+    ml_parts = torch.randn((R_m, w.B, w.Hq, w.Nq), generator=g_m).to(dev)
+    m_out = torch.empty((w.B, w.Nq, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
+    m_lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=dev)
+
+    def merge():
+        ea.attn_merge(mo_parts, ml_parts, o=m_out, lse=m_lse)
+
+    mtimes, mlaunches = timed_kernel_loop(merge, args.steps, args.warmup, world, None, None)
+    mms = statistics.mean(mtimes)
+    mms_max = max_over_ranks(mms, world)
+    m_rows = w.B * w.Nq * w.Hq
+    m_bytes = R_m * m_rows * (w.d + 1) * 4 + m_rows * (w.d * 2 + 4)
+    m_value = whole_job_rate(m_bytes, mms_max, world) / 1e9
+    m_achieved = m_bytes / (mms * 1e-3) / 1e9
+    del mo_parts, ml_parts, m_out, m_lse
+
     # packed variable-length prefill leg: 16 causal sequences with seeded
     # lengths in [256, 4096], MHA H32 d128, no padding
     vl_lens = ai.varlen_lengths(16, 256, 4096, seed=shard_seed(rank) + 13)
@@ -539,6 +561,15 @@ def run_ours(args, world, rank, local):
                          "kernel": "bwd_prep_kernel + bwd_main_kernel<128> + bwd_finalize_kernel",
                          "traffic": None},
             "gpu_launches": blaunches,
+        },
+        "merge": {
+            "workload": f"merge of {R_m} fp32 parts, {w.name} output shape", "value": m_value,
+            "unit": "GB/s", "ms_per_step": mms_max,
+            "roofline": {"bound": "hbm", "achieved": m_achieved, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": m_achieved / peaks["hbm_gbs"],
+                         "peak_source": f"{peak_src} hbm_gbs", "kernel": "attn_merge_kernel<128>",
+                         "algorithmic_bytes": m_bytes, "traffic": None},
+            "gpu_launches": mlaunches,
         },
         "varlen": {
             "workload": f"MHA causal packed prefill, 16 sequences of {min(vl_lens)}-{max(vl_lens)} "

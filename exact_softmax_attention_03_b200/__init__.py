@@ -20,7 +20,7 @@ import torch
 from ._lib import AttnError, check, load  # noqa: F401
 
 __all__ = ["attn_fwd", "attn_fwd_f32o", "attn_fwd_varlen", "attn_bwd", "attn_bwd_workspace_bytes",
-           "attn_decode", "attn_decode_paged",
+           "attn_merge", "attn_decode", "attn_decode_paged",
            "attn_decode_workspace_bytes", "attn_decode_noalloc",
            "attn_device_status", "attn_last_error", "attn_launch_count", "AttnError"]
 
@@ -156,6 +156,25 @@ def attn_bwd(q, k, v, o, lse, dout, causal=False, window_left=-1, scale=None, dq
                           Nq, Nk, d, float(scale), int(bool(causal)), int(window_left),
                           workspace.data_ptr(), ws_bytes, _stream_handle(stream)))
     return dq, dk, dv
+
+
+def attn_merge(o_parts, lse_parts, o=None, lse=None, stream=None):
+    """Merge per-key-shard results. ``o_parts [R, B, Nq, Hq, d]`` f32 and
+    ``lse_parts [R, B, Hq, Nq]`` f32 (CUDA). Returns ``(o bf16 [B, Nq, Hq, d], lse)``."""
+    _need(o_parts, "o_parts", torch.float32, 5)
+    _need(lse_parts, "lse_parts", torch.float32, 4)
+    R, B, Nq, Hq, d = o_parts.shape
+    if tuple(lse_parts.shape) != (R, B, Hq, Nq):
+        raise ValueError("lse_parts must be [R, B, Hq, Nq] matching o_parts")
+    if o is None:
+        o = torch.empty((B, Nq, Hq, d), dtype=torch.bfloat16, device=o_parts.device)
+    _need(o, "o", torch.bfloat16, 4)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, 3)
+    check(load().attn_merge(o_parts.data_ptr(), lse_parts.data_ptr(), R, o.data_ptr(),
+                            lse.data_ptr() if lse is not None else None, B, Nq, Hq, d,
+                            _stream_handle(stream)))
+    return o, lse
 
 
 def attn_decode_workspace_bytes(B: int, Hq: int, d: int, num_splits: int = 0, Lmax: int = 1) -> int:

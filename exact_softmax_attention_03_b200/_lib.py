@@ -40,6 +40,7 @@ SIGNATURES = {
     "attn_bwd_workspace_bytes": (ctypes.c_size_t, [_i, _i, _i, _i]),
     "attn_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i,
                       _i, _vp, ctypes.c_size_t, _vp]),
+    "attn_merge": (_i, [_vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _vp]),
     "attn_decode_workspace_bytes": (ctypes.c_size_t, [_i, _i, _i, _i, _i]),
     "attn_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _i, _vp,
                          ctypes.c_size_t, _vp]),

@@ -17,7 +17,7 @@ ROOT = os.path.dirname(HERE)
 SRC = os.path.join(HERE, "csrc", "attn_api.cu")
 DEPS = [os.path.join(HERE, "csrc", f) for f in
         ("attn_api.cu", "sm100_ptx.cuh", "decode_kernels.cuh", "prefill_kernel.cuh",
-         "backward_kernels.cuh")] + \
+         "backward_kernels.cuh", "merge_kernel.cuh")] + \
        [os.path.join(ROOT, "include", "attn.h")]
 LIB = os.path.join(HERE, "libattn.so")
 

@@ -1,0 +1,69 @@
+"""Sequence-sharded (context-parallel) attention over torch.distributed.
+
+Each rank holds one equal-length chunk of the sequence: its queries and its
+keys/values. The ranks all-gather the K/V chunks (NCCL over NVLink between
+GPUs), each rank attends its query chunk to every chunk it may see with the
+library's forward kernel, and the per-chunk results are merged with the
+rescale-to-common-maximum rule ("Chapter 3: MHA Limitations, MQA, GQA, and
+FlashAttention", section 3.5) by the library's merge kernel. The use is the
+long-context case of "How to Reduce Attention Computation Cost in LLM
+Training", section "Ring Attention and Sequence Parallelism": when one GPU's
+memory is the wall, the sequence is split across NVLink-connected GPUs.
+
+Causal masking across chunks: rank r's queries sit at global positions
+[r*C, (r+1)*C); chunk s < r is wholly visible, chunk r is the usual causal
+(diagonal) block, chunks s > r are wholly masked and skipped. Sliding windows
+are not supported here. All arithmetic runs in the library's kernels; this
+module only moves tensors and chooses calls.
+"""
+
+from __future__ import annotations
+
+import torch
+
+from . import attn_fwd_f32o, attn_merge
+
+
+def chunk_plan(rank: int, world: int, causal: bool):
+    """``[(s, is_causal_block)]``: the K/V chunks rank ``rank`` attends to."""
+    if not 0 <= rank < world:
+        raise ValueError("rank out of range")
+    if not causal:
+        return [(s, False) for s in range(world)]
+    return [(s, s == rank) for s in range(rank + 1)]
+
+
+def gather_chunks(x: torch.Tensor, group=None) -> list:
+    """All-gather one equal-shaped chunk per rank; returns the list in rank order."""
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    out = [torch.empty_like(x) for _ in range(world)]
+    dist.all_gather(out, x.contiguous(), group=group)
+    return out
+
+
+def context_parallel_local(q, k_chunks, v_chunks, rank: int, causal: bool = True, scale=None,
+                           lse=None):
+    """Attention of this rank's query chunk ``q [B, C, Hq, d]`` to the gathered
+    K/V chunks (``[B, C, Hkv, d]`` each, rank order). Returns ``(o, lse)``."""
+    world = len(k_chunks)
+    plan = chunk_plan(rank, world, causal)
+    B, C, Hq, d = q.shape
+    o_parts = torch.empty((len(plan), B, C, Hq, d), dtype=torch.float32, device=q.device)
+    lse_parts = torch.empty((len(plan), B, Hq, C), dtype=torch.float32, device=q.device)
+    for i, (s, diag) in enumerate(plan):
+        attn_fwd_f32o(q, k_chunks[s], v_chunks[s], o=o_parts[i], lse=lse_parts[i], causal=diag,
+                      scale=scale)
+    if lse is None:
+        lse = torch.empty((B, Hq, C), dtype=torch.float32, device=q.device)
+    return attn_merge(o_parts, lse_parts, lse=lse)
+
+
+def context_parallel_attention(q, k, v, group=None, causal: bool = True, scale=None):
+    """Sequence-sharded attention: each rank passes its own chunk of Q, K, V
+    (equal lengths on every rank); returns this rank's chunk of O and LSE."""
+    import torch.distributed as dist
+    rank = dist.get_rank(group)
+    k_chunks = gather_chunks(k, group)
+    v_chunks = gather_chunks(v, group)
+    return context_parallel_local(q, k_chunks, v_chunks, rank, causal=causal, scale=scale)

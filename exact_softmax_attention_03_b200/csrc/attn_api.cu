@@ -12,10 +12,12 @@
 #include <cstring>
 #include <algorithm>
 #include <mutex>
+#include <type_traits>
 
 #include "../../include/attn.h"
 #include "backward_kernels.cuh"
 #include "decode_kernels.cuh"
+#include "merge_kernel.cuh"
 #include "prefill_kernel.cuh"
 
 namespace {
@@ -518,6 +520,46 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const v
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "attn_bwd launch: %s", cudaGetErrorString(e));
   g_launches.fetch_add(3);
+  return ok();
+}
+
+int attn_merge(const float* o_parts, const float* lse_parts, int R, void* o, float* lse, int B,
+               int Nq, int Hq, int d, cudaStream_t stream) {
+  if (!o_parts || !lse_parts || !o)
+    return fail(ATTN_ERR_INVALID_ARG, "o_parts, lse_parts and o must be non-null");
+  if (R < 1 || B < 1 || Nq < 1 || Hq < 1)
+    return fail(ATTN_ERR_INVALID_ARG, "R, B, Nq, Hq must be >= 1");
+  if (R > 64) return fail(ATTN_ERR_UNSUPPORTED, "at most 64 parts (got %d)", R);
+  if (d != 64 && d != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim %d not in {64, 128}", d);
+  if (!aligned(o_parts, 16) || !aligned(o, 8) || !aligned(lse_parts, 4) || (lse && !aligned(lse, 4)))
+    return fail(ATTN_ERR_INVALID_ARG, "o_parts must be 16-byte, o 8-byte, lse 4-byte aligned");
+  const long long rows = static_cast<long long>(B) * Nq * Hq;
+  if (rows * d > kMaxIndex * 16ll || rows * R > kMaxIndex * 16ll)
+    return fail(ATTN_ERR_INVALID_ARG, "sizes too large");
+  int dev = 0;
+  int rc = check_device(&dev);
+  if (rc != ATTN_OK) return rc;
+  const unsigned grid = unsigned((rows * 32 + 255) / 256);
+  uint16_t* ob = static_cast<uint16_t*>(o);
+  // part count rounded up to a compile-time bound: all loads go out at once
+  auto go = [&](auto dtag, auto rtag) {
+    constexpr int DD = decltype(dtag)::value, RR = decltype(rtag)::value;
+    attn::attn_merge_kernel<DD, RR><<<grid, 256, 0, stream>>>(o_parts, lse_parts, R, ob, lse, B, Nq, Hq);
+  };
+  using D128 = std::integral_constant<int, 128>;
+  using D64 = std::integral_constant<int, 64>;
+  auto by_r = [&](auto dtag) {
+    if (R <= 2) go(dtag, std::integral_constant<int, 2>{});
+    else if (R <= 4) go(dtag, std::integral_constant<int, 4>{});
+    else if (R <= 8) go(dtag, std::integral_constant<int, 8>{});
+    else if (R <= 16) go(dtag, std::integral_constant<int, 16>{});
+    else go(dtag, std::integral_constant<int, 64>{});
+  };
+  if (d == 128) by_r(D128{});
+  else by_r(D64{});
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "attn_merge launch: %s", cudaGetErrorString(e));
+  g_launches.fetch_add(1);
   return ok();
 }
 

@@ -132,6 +132,24 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const v
              size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * Merge attention results computed over disjoint key sets (for example the
+ * key shards of sequence-sharded attention): per query row, each part r has a
+ * normalised output O_r and its log-sum-exp LSE_r; the merged result rescales
+ * the parts to the common maximum before adding ("Chapter 3: MHA Limitations,
+ * MQA, GQA, and FlashAttention", section 3.5): M = max LSE_r,
+ * w_r = exp(LSE_r - M), O = sum w_r O_r / sum w_r, LSE = M + ln sum w_r.
+ * A row no part saw a key for (every LSE_r = -inf) gets O = 0, LSE = -inf.
+ *   o_parts   : device f32 [R, B, Nq, Hq, d], 16-byte aligned
+ *   lse_parts : device f32 [R, B, Hq, Nq]
+ *   o         : device bf16 [B, Nq, Hq, d], 8-byte aligned (written)
+ *   lse       : device f32 [B, Hq, Nq] or NULL
+ *   1 <= R <= 64; B, Nq, Hq >= 1; d in {64, 128}
+ * Returns ATTN_OK or an attn_status; nothing is launched on error.
+ */
+int attn_merge(const float* o_parts, const float* lse_parts, int R, void* o, float* lse, int B,
+               int Nq, int Hq, int d, cudaStream_t stream);
+
+/*
  * Bytes of device workspace attn_decode needs for these sizes.
  * num_splits = 0 picks the split count attn_decode would pick automatically.
  * Returns 0 for invalid sizes.

@@ -33,7 +33,7 @@ def header_functions():
 def test_header_declares_the_expected_entry_points():
     assert header_functions() == sorted([
         "attn_fwd", "attn_fwd_f32o", "attn_fwd_varlen", "attn_bwd", "attn_bwd_workspace_bytes",
-        "attn_decode_workspace_bytes",
+        "attn_decode_workspace_bytes", "attn_merge",
         "attn_decode",
         "attn_decode_paged", "attn_decode_noalloc", "attn_last_error", "attn_device_status",
         "attn_launch_count",

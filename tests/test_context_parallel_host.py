@@ -1,0 +1,61 @@
+"""Host logic of sequence-sharded attention (CPU): which K/V chunks each rank
+attends to, and the all-gather that assembles them, run as two gloo ranks."""
+
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from exact_softmax_attention_03_b200.context_parallel import chunk_plan
+
+
+def test_chunk_plan_causal_and_full():
+    assert chunk_plan(0, 4, True) == [(0, True)]
+    assert chunk_plan(2, 4, True) == [(0, False), (1, False), (2, True)]
+    assert chunk_plan(3, 4, False) == [(0, False), (1, False), (2, False), (3, False)]
+    # every (query chunk, key chunk) pair with an allowed key is covered exactly once
+    world = 5
+    pairs = {(r, s) for r in range(world) for s, _ in chunk_plan(r, world, True)}
+    assert pairs == {(r, s) for r in range(world) for s in range(world) if s <= r}
+    with pytest.raises(ValueError):
+        chunk_plan(4, 4, True)
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port),
+                      RANK=str(rank), WORLD_SIZE=str(world))
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        from exact_softmax_attention_03_b200.context_parallel import gather_chunks
+        x = torch.full((2, 3, 1, 4), float(rank + 1))
+        chunks = gather_chunks(x)
+        out.put((rank, [float(c[0, 0, 0, 0]) for c in chunks], [tuple(c.shape) for c in chunks]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_gather_chunks_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in range(2))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, vals, shapes in res:
+        assert vals == [1.0, 2.0]                    # rank order on every rank
+        assert shapes == [(2, 3, 1, 4)] * 2
