@@ -178,6 +178,21 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     p.n_bh = B * Hq;
   }
   p.nbh_seq = p.n_bh / B;
+  p.vl_hg = p.nbh_seq;
+  if (pk) {
+    // Head groups for the packed work list: the largest divisor of the items per
+    // (sequence, unit) for which the K/V the concurrently running items touch
+    // (estimated from the average sequence) stays within 96 MB of L2.
+    const double kv_per_seq_head = double(pk->total_k) / B * D * 2.0 * 2.0;
+    const int items_per_kv_head = p.nbh_seq / Hkv;
+    for (int hg = p.nbh_seq; hg >= 1; --hg) {
+      if (p.nbh_seq % hg) continue;
+      const double live = std::min(148.0, double(B) * hg);     // items running at once
+      const double kv_heads = std::max(1.0, live / items_per_kv_head);
+      p.vl_hg = hg;
+      if (kv_heads * kv_per_seq_head <= 96.0 * (1 << 20)) break;
+    }
+  }
   const long long items = static_cast<long long>(p.n_units) * p.n_bh;
   if (items > kMaxIndex) return fail(ATTN_ERR_INVALID_ARG, "problem too large for one launch");
   if (pk && (B > L::VL_MAX_SEQS || p.n_units > L::VL_MAX_UNITS))

@@ -99,6 +99,7 @@ struct FwdParams {
   const int* cu_k;
   int total_q, total_k;
   int nbh_seq;             // items per (sequence, row unit): n_bh / B
+  int vl_hg;               // packed: heads (or head pairs) per group, divides nbh_seq
   int causal, window_left;
   float scale;             // softmax scale
   float scale_log2;        // scale * log2(e)
@@ -205,10 +206,13 @@ struct WorkItem {
   int ubhi, U;             // key blocks visited: ubhi-1 down to ubhi-U
 };
 
-// Packed sequences: the work list holds only the items that exist, longest
-// rows first. Sequences are sorted by their number of row units (descending),
-// so at unit level u the sequences with more than u units are a prefix
-// perm[0 .. cnt[u]) of the sorted order; level u's items start at lvl[u].
+// Packed sequences: the work list holds only the items that exist. The heads
+// (or head pairs) are taken in groups of vl_hg, one group after another, so the
+// K/V of the items running at once fits in L2; within a group the rows run
+// longest first. Sequences are sorted by their number of row units
+// (descending), so at unit level u the sequences with more than u units are a
+// prefix perm[0 .. cnt[u]) of the sorted order; level u's items start at
+// lvl[u] within the group, and lvl[n_units] is the size of a group.
 
 __device__ __forceinline__ int varlen_valid_rows(const FwdParams& p, int b) {
   const int q0 = __ldg(p.cu_q + b), q1 = __ldg(p.cu_q + b + 1);
@@ -232,7 +236,7 @@ __device__ void build_varlen_sched(const FwdParams& p, int* vl, int* n_items) {
   int* lvl = vl + kVlLvl;
   int* cur = vl + kVlCur;
   const int U = p.n_units;
-  const int nbh = p.nbh_seq;                             // items per (sequence, unit)
+  const int hg = p.vl_hg;                                // items per (sequence, unit, group)
   for (int u = threadIdx.x; u <= U; u += blockDim.x) cnt[u] = 0;
   __syncthreads();
   for (int b = threadIdx.x; b < p.B; b += blockDim.x) {
@@ -251,12 +255,14 @@ __device__ void build_varlen_sched(const FwdParams& p, int* vl, int* n_items) {
       cur[v] = slot;
       slot += h;
     }
+    // levels within one head group; the groups repeat the pattern
     int item = 0;
     for (int u = U - 1; u >= 0; --u) {
       lvl[u] = item;
-      item += cnt[u] * nbh;
+      item += cnt[u] * hg;
     }
-    *n_items = item;
+    lvl[U] = item;                                       // items of one head group
+    *n_items = item * (p.nbh_seq / hg);
   }
   __syncthreads();
   for (int b = threadIdx.x; b < p.B; b += blockDim.x)
@@ -271,16 +277,20 @@ __device__ __forceinline__ void decode_item(const FwdParams& p, int item, WorkIt
   int unit, bh;
   if constexpr (VARLEN) {
     const int* lvl = vl + kVlLvl;
-    // level: the lowest u whose first item is <= item (lvl grows as u falls)
+    // head group, then level: the lowest u whose first item is <= the item's
+    // index within the group (lvl grows as u falls)
+    const int per_group = lvl[p.n_units];
+    const int g = item / per_group;
+    const int ig = item - g * per_group;
     int lo = 0, hi = p.n_units - 1;
     while (lo < hi) {
       const int mid = (lo + hi) >> 1;
-      if (lvl[mid] <= item) hi = mid; else lo = mid + 1;
+      if (lvl[mid] <= ig) hi = mid; else lo = mid + 1;
     }
     unit = lo;
-    const int r = item - lvl[unit];
-    const int s = r / p.nbh_seq;
-    bh = vl[s] * p.nbh_seq + (r - s * p.nbh_seq);
+    const int r = ig - lvl[unit];
+    const int s = r / p.vl_hg;
+    bh = vl[s] * p.nbh_seq + g * p.vl_hg + (r - s * p.vl_hg);
   } else {
     unit = p.n_units - 1 - item / p.n_bh;                // longest rows first
     bh = item % p.n_bh;
