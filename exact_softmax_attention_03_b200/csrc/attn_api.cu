@@ -382,6 +382,9 @@ template <int D>
 int launch_bwd(const void* q, const void* k, const void* v, attn::BwdParams& p, cudaStream_t stream,
                int dev) {
   using L = attn::BwdLayout<D>;
+  const long long nbh = static_cast<long long>(p.B) * p.Hkv;
+  const long long nctas = static_cast<long long>((p.Nk + 127) / 128) * nbh;
+  if (nctas > kMaxIndex) return fail(ATTN_ERR_INVALID_ARG, "problem too large for one launch");
   CUtensorMap mq, mk, mv, mdo;
   int rc;
   if ((rc = make_map(&mq, q, D, p.Hq, p.Nq, p.B)) != ATTN_OK) return rc;
@@ -398,10 +401,13 @@ int launch_bwd(const void* q, const void* k, const void* v, attn::BwdParams& p, 
   }
   const long long rows = static_cast<long long>(p.B) * p.Nq * p.Hq;
   attn::bwd_prep_kernel<D><<<unsigned((rows * 32 + 255) / 256), 256, 0, stream>>>(p);
-  const dim3 grid(unsigned((p.Nk + 127) / 128), unsigned(p.Hkv), unsigned(p.B));
-  attn::bwd_main_kernel<D><<<grid, attn::kBwdThreads, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, p);
-  const long long n8 = rows * D / 8;
-  attn::bwd_finalize_kernel<<<unsigned((n8 + 255) / 256), 256, 0, stream>>>(p, n8);
+  // chunk of (batch, K/V head) pairs whose Q, dO (bf16) and dQ accumulator
+  // (fp32) rows take about 48 MB of L2
+  const long long unit = static_cast<long long>(p.Hq / p.Hkv) * p.Nq * D * 8;
+  p.bh_chunk = static_cast<int>(std::max(1ll, std::min(nbh, (48ll << 20) / unit)));
+  attn::bwd_main_kernel<D><<<unsigned(nctas), attn::kBwdThreads, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, p);
+  const long long fin = static_cast<long long>(p.B) * p.Hq * ((p.Nq + attn::kFinQ - 1) / attn::kFinQ);
+  attn::bwd_finalize_kernel<D><<<unsigned(fin), 256, 0, stream>>>(p);
   return ATTN_OK;
 }
 

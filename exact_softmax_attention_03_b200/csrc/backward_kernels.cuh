@@ -22,6 +22,7 @@
 //              a query row (reading dQ); at the end a key row again (dK, dV)
 //   warp 4     tensor-core issuer (whole warp, one elected lane issues)
 //   warp 5     TMA producer (one lane): K_j, V_j once; Q_i, dO_i per block
+//              through a 2-stage ring (the next block's tiles load during this one)
 // Per query block (tile = 128 x 128):
 //   Sᵀ  = K_j Q_iᵀ        SS, both K-major                 -> TMEM cols [0,128)
 //   dPᵀ = V_j dO_iᵀ       SS, both K-major                 -> TMEM cols [128,256)
@@ -52,13 +53,14 @@ struct BwdParams {
   const uint16_t* dout;    // [B, Nq, Hq, D] bf16
   const float* lse;        // [B, Hq, Nq] natural log-sum-exp of the forward
   float* delta;            // [B, Hq, Nq] rowsum(dO * O)              (workspace)
-  float* dq_acc;           // [B, Nq, Hq, D] fp32, scale * dQ         (workspace)
+  float* dq_acc;           // [B, Hq, D/4, Nq] float4, scale * dQ     (workspace)
   uint16_t* dq;            // [B, Nq, Hq, D] bf16
   uint16_t* dk;            // [B, Nk, Hkv, D] bf16
   uint16_t* dv;            // [B, Nk, Hkv, D] bf16
   int B, Hq, Hkv, Nq, Nk;
   int causal, window_left;
   float scale, scale_log2;
+  int bh_chunk;            // (batch, K/V head) pairs per scheduling chunk, >= 1
 };
 
 // ---- delta = rowsum(dO * O); zero the dQ accumulator ------------------------
@@ -82,7 +84,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p) {
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
 #pragma unroll
-  for (int e = 0; e < EPL; ++e) p.dq_acc[base + e] = 0.f;
+  for (int e = 0; e < EPL; ++e) p.dq_acc[base + e] = 0.f;   // slice `row` of the buffer
   if (lane == 0) {
     const int h = int(row % p.Hq);
     const long long bq = row / p.Hq;                         // b * Nq + q
@@ -93,17 +95,39 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p) {
 }
 
 // ---- dQ accumulator (already scaled) -> bf16 --------------------------------
-__global__ void __launch_bounds__(256) bwd_finalize_kernel(const BwdParams p, long long n8) {
-  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= n8) return;
-  const float4 a = reinterpret_cast<const float4*>(p.dq_acc)[2 * i];
-  const float4 b = reinterpret_cast<const float4*>(p.dq_acc)[2 * i + 1];
-  uint4 v;
-  v.x = pack_bf16x2(a.x, a.y);
-  v.y = pack_bf16x2(a.z, a.w);
-  v.z = pack_bf16x2(b.x, b.y);
-  v.w = pack_bf16x2(b.z, b.w);
-  reinterpret_cast<uint4*>(p.dq)[i] = v;
+// The accumulator keeps each 4-wide column chunk of a (batch, head) contiguous
+// over the queries, so that a warp's atomics (32 consecutive queries) cover
+// 512 contiguous bytes. One CTA turns 64 queries of one (batch, head) back
+// into rows of dq through shared memory: reads and writes both coalesced.
+constexpr int kFinQ = 64;
+
+template <int D>
+__global__ void __launch_bounds__(256) bwd_finalize_kernel(const BwdParams p) {
+  constexpr int C4 = D / 4;
+  __shared__ float4 tile[C4][kFinQ + 1];
+  const int nqt = (p.Nq + kFinQ - 1) / kFinQ;
+  const long long bh = static_cast<long long>(blockIdx.x) / nqt;      // b * Hq + hq
+  const int q0 = int(static_cast<long long>(blockIdx.x) % nqt) * kFinQ;
+  const float4* src = reinterpret_cast<const float4*>(p.dq_acc) + size_t(bh) * C4 * p.Nq;
+  for (int idx = threadIdx.x; idx < C4 * kFinQ; idx += blockDim.x) {
+    const int c = idx / kFinQ, ql = idx % kFinQ;
+    const int q = q0 + ql;
+    tile[c][ql] = q < p.Nq ? src[size_t(c) * p.Nq + q] : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  __syncthreads();
+  const int hq = int(bh % p.Hq), b = int(bh / p.Hq);
+  for (int idx = threadIdx.x; idx < kFinQ * (D / 8); idx += blockDim.x) {
+    const int ql = idx / (D / 8), g = idx % (D / 8);
+    const int q = q0 + ql;
+    if (q >= p.Nq) continue;
+    const float4 a = tile[2 * g][ql], c = tile[2 * g + 1][ql];
+    uint4 v;
+    v.x = pack_bf16x2(a.x, a.y);
+    v.y = pack_bf16x2(a.z, a.w);
+    v.z = pack_bf16x2(c.x, c.y);
+    v.w = pack_bf16x2(c.z, c.w);
+    reinterpret_cast<uint4*>(p.dq + ((size_t(b) * p.Nq + q) * p.Hq + hq) * D)[g] = v;
+  }
 }
 
 template <int D>
@@ -112,21 +136,21 @@ struct BwdLayout {
   static constexpr int HALF = 128 * 128;                   // 128 rows x 64 columns, swizzled
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + TILE;
-  static constexpr int OFF_Q = OFF_V + TILE;
-  static constexpr int OFF_DO = OFF_Q + TILE;
-  static constexpr int OFF_DS = OFF_DO + TILE;             // dSᵀ [128 keys][128 queries] bf16
-  static constexpr int OFF_LD = OFF_DS + 2 * HALF;         // f32 lse2[2][128], delta[2][128]
-  static constexpr int OFF_BAR = OFF_LD + 4 * 128 * 4;
+  static constexpr int OFF_Q = OFF_V + TILE;              // Q_i, 2 stages
+  static constexpr int OFF_DO = OFF_Q + 2 * TILE;          // dO_i, 2 stages
+  static constexpr int OFF_DS = OFF_DO + 2 * TILE;         // dSᵀ [128 keys][128 queries] bf16
+  static constexpr int OFF_LD = OFF_DS + 2 * HALF;         // f32 lse2[128], delta[128]
+  static constexpr int OFF_BAR = OFF_LD + 2 * 128 * 4;
   static constexpr int B_KV = 0;     // K_j, V_j loaded
-  static constexpr int B_QD = 1;     // Q_i, dO_i loaded
-  static constexpr int B_QDE = 2;    // Q_i, dO_i and the dS tile free again
-  static constexpr int B_SD = 3;     // Sᵀ and dPᵀ in TMEM
-  static constexpr int B_PR = 4;     // Pᵀ, dSᵀ written (128 arrivals)
-  static constexpr int B_QR = 5;     // dQ_i in TMEM
-  static constexpr int B_QF = 6;     // dQ_i read (128 arrivals)
-  static constexpr int B_DONE = 7;   // every dK / dV product complete
-  static constexpr int B_LD = 8;     // per-block lse2 / delta values in shared memory (128 arrivals)
-  static constexpr int NBAR = 9;
+  static constexpr int B_QD = 1;     // Q_i, dO_i loaded, + stage
+  static constexpr int B_QDE = 3;    // Q_i, dO_i stage free again, + stage
+  static constexpr int B_SD = 5;     // Sᵀ and dPᵀ in TMEM
+  static constexpr int B_PR = 6;     // Pᵀ, dSᵀ written (128 arrivals)
+  static constexpr int B_QR = 7;     // dQ_i in TMEM
+  static constexpr int B_QF = 8;     // dQ_i read (128 arrivals)
+  static constexpr int B_DONE = 9;   // every dK / dV product complete
+  static constexpr int B_LD = 10;    // per-block lse2 / delta values in shared memory (128 arrivals)
+  static constexpr int NBAR = 11;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;      // [0] TMEM base, [1] abort flag
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = BYTES + 1024;
@@ -166,7 +190,18 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  const int j = blockIdx.x, hkv = blockIdx.y, b = blockIdx.z;
+  // One CTA per (batch, K/V head, 128-key block) on a 1-D grid. The (batch,
+  // head) pairs go in chunks of bh_chunk, whose Q, dO and dQ rows stay in L2
+  // together; inside a chunk the key blocks run heaviest first (most query
+  // blocks), so the last CTAs to start are the short ones.
+  const int nkb = (p.Nk + 127) / 128, nbh = p.B * p.Hkv;
+  const int per_chunk = p.bh_chunk * nkb;
+  const int chunk = int(blockIdx.x) / per_chunk, r = int(blockIdx.x) % per_chunk;
+  const int cs = min(p.bh_chunk, nbh - chunk * p.bh_chunk);
+  const int jj = r / cs, bh = chunk * p.bh_chunk + r % cs;
+  // causal: earlier key blocks see more queries; window only: later ones do
+  const int j = (p.causal || p.window_left < 0) ? jj : nkb - 1 - jj;
+  const int hkv = bh % p.Hkv, b = bh / p.Hkv;
   const int G = p.Hq / p.Hkv;
   const int kb0 = j * 128, kb1 = min(kb0 + 127, p.Nk - 1);
   int i_lo, i_hi;
@@ -176,8 +211,10 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
   if (threadIdx.x == 0) {
     mbar_init(bar(L::B_KV), 1);
-    mbar_init(bar(L::B_QD), 1);
-    mbar_init(bar(L::B_QDE), 1);
+    for (int st = 0; st < 2; ++st) {
+      mbar_init(bar(L::B_QD + st), 1);
+      mbar_init(bar(L::B_QDE + st), 1);
+    }
     mbar_init(bar(L::B_SD), 1);
     mbar_init(bar(L::B_PR), 128);
     mbar_init(bar(L::B_QR), 1);
@@ -201,8 +238,11 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const int t = int(threadIdx.x);                          // TMEM lane
     const uint32_t lane_off = uint32_t(warp * 32) << 16;
     const uint32_t tST = tmem + lane_off + L::COL_ST, tDPT = tmem + lane_off + L::COL_DPT;
-    float* lse2_s = reinterpret_cast<float*>(smem + L::OFF_LD);          // [2][128]
-    float* delta_s = lse2_s + 2 * 128;                                   // [2][128]
+    // one buffer is enough: block n's values are stored only after B_SD(n),
+    // whose products were issued after every thread arrived on B_QF(n-1),
+    // i.e. after every read of block n-1's values
+    float* lse2_s = reinterpret_cast<float*>(smem + L::OFF_LD);          // [128]
+    float* delta_s = lse2_s + 128;                                       // [128]
     const int key = kb0 + t;
     const int off = p.Nk - p.Nq;
     const float c2 = p.scale_log2;
@@ -211,16 +251,19 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const int g = n / nblk, i = i_lo + n % nblk;
       const int hq = hkv * G + g;
       const int par = n & 1;
+      float l2v, dv;
       {
         const int q = i * 128 + t;
         const bool qv = q < p.Nq;
         const float l = qv ? __ldg(p.lse + (size_t(b) * p.Hq + hq) * p.Nq + q) : 0.f;
-        lse2_s[par * 128 + t] = (qv && l > -CUDART_INF_F) ? l * 1.4426950408889634f : 0.f;
-        delta_s[par * 128 + t] = qv ? __ldg(p.delta + (size_t(b) * p.Hq + hq) * p.Nq + q) : 0.f;
+        l2v = (qv && l > -CUDART_INF_F) ? l * 1.4426950408889634f : 0.f;
+        dv = qv ? __ldg(p.delta + (size_t(b) * p.Hq + hq) * p.Nq + q) : 0.f;
       }
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_SD), uint32_t(par), abort_flag)))) break;
+      lse2_s[t] = l2v;
+      delta_s[t] = dv;
       mbar_arrive(bar(L::B_LD));
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_LD), uint32_t(par), abort_flag)))) break;
-      if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_SD), uint32_t(par), abort_flag)))) break;
       tc_fence_after();
       // allowed queries of this key within the block: [c_lo, c_hi]
       const int q0 = i * 128;
@@ -228,8 +271,8 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       if (key >= p.Nk) c_hi = -1;
       if (p.causal) c_lo = max(c_lo, key - off - q0);                    // key <= q + off
       if (p.window_left >= 0) c_hi = min(c_hi, key + p.window_left - off - q0);
-      const float* lsr = lse2_s + par * 128;
-      const float* dlt = delta_s + par * 128;
+      const float* lsr = lse2_s;
+      const float* dlt = delta_s;
       // 64 queries at a time: read their Sᵀ and dPᵀ columns (32 at a time),
       // then write the bf16 pairs of Pᵀ and dSᵀ over columns already read
 #pragma unroll
@@ -288,10 +331,11 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       mbar_arrive(bar(L::B_QF));
       const int q = q0 + t;
       if (q < p.Nq) {
-        float4* dst = reinterpret_cast<float4*>(p.dq_acc + ((size_t(b) * p.Nq + q) * p.Hq + hq) * D);
+        // chunk e of query q: the warp's 32 queries are 32 adjacent float4
+        float4* dst = reinterpret_cast<float4*>(p.dq_acc) + (size_t(b) * p.Hq + hq) * (D / 4) * p.Nq + q;
 #pragma unroll
         for (int e = 0; e < D / 4; ++e)
-          atomicAdd(dst + e, make_float4(__uint_as_float(qr[4 * e]) * p.scale,
+          atomicAdd(dst + size_t(e) * p.Nq, make_float4(__uint_as_float(qr[4 * e]) * p.scale,
                                          __uint_as_float(qr[4 * e + 1]) * p.scale,
                                          __uint_as_float(qr[4 * e + 2]) * p.scale,
                                          __uint_as_float(qr[4 * e + 3]) * p.scale));
@@ -351,19 +395,21 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     bool alive = total > 0 && wwait(L::B_KV, 0u);
     for (int n = 0; alive && n < total; ++n) {
       const uint32_t par = uint32_t(n & 1);
-      if (!(alive = wwait(L::B_QD, par))) break;
+      const int stg = n & 1;                                     // Q/dO stage of this block
+      const uint32_t so = uint32_t(stg * (L::TILE >> 4));       // its descriptor offset
+      if (!(alive = wwait(L::B_QD + stg, uint32_t((n >> 1) & 1)))) break;
       if (n > 0 && !(alive = wwait(L::B_QF, par ^ 1u))) break;   // previous dQ read out
       tc_fence_after();
       // Sᵀ = K_j Q_iᵀ and dPᵀ = V_j dO_iᵀ (K = d)
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
         const uint32_t o = ((k / 4) * L::HALF + (k % 4) * 32) >> 4;
-        if (elect_one()) mma_ss(tST, dK_k + o, dQ_k + o, L::IDESC_S, k > 0 ? 1u : 0u);
+        if (elect_one()) mma_ss(tST, dK_k + o, dQ_k + so + o, L::IDESC_S, k > 0 ? 1u : 0u);
       }
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
         const uint32_t o = ((k / 4) * L::HALF + (k % 4) * 32) >> 4;
-        if (elect_one()) mma_ss(tDPT, dV_k + o, dO_k + o, L::IDESC_S, k > 0 ? 1u : 0u);
+        if (elect_one()) mma_ss(tDPT, dV_k + o, dO_k + so + o, L::IDESC_S, k > 0 ? 1u : 0u);
       }
       commit(L::B_SD);
       if (!(alive = wwait(L::B_PR, par))) break;
@@ -372,12 +418,12 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
         const uint32_t o = (k * 16 * 128) >> 4;
-        if (elect_one()) mma_ts(tDV, tST + 8 * k, dO_mn + o, L::IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
+        if (elect_one()) mma_ts(tDV, tST + 8 * k, dO_mn + so + o, L::IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
       }
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
         const uint32_t o = (k * 16 * 128) >> 4;
-        if (elect_one()) mma_ts(tDK, tDPT + 8 * k, dQ_mn + o, L::IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
+        if (elect_one()) mma_ts(tDK, tDPT + 8 * k, dQ_mn + so + o, L::IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
       }
       // dQ_i = dS K_j, 64 columns of d at a time (K = 128 keys)
 #pragma unroll
@@ -391,7 +437,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         }
       }
       commit(L::B_QR);
-      commit(L::B_QDE);
+      commit(L::B_QDE + stg);
     }
     if (total > 0) {
       commit(L::B_DONE);                        // also drains every issued product
@@ -414,17 +460,22 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       for (int n = 0; n < total; ++n) {
         const int g = n / nblk, i = i_lo + n % nblk;
         const int hq = hkv * G + g;
-        if (n > 0 && !mbar_wait(bar(L::B_QDE), uint32_t((n - 1) & 1), abort_flag)) break;
-        mbar_arrive_expect_tx(bar(L::B_QD), 2 * L::TILE);
+        const int stg = n & 1;
+        // the stage is free once the products of block n - 2 completed
+        if (n >= 2 && !mbar_wait(bar(L::B_QDE + stg), uint32_t(((n >> 1) - 1) & 1), abort_flag)) break;
+        mbar_arrive_expect_tx(bar(L::B_QD + stg), 2 * L::TILE);
         for (int c = 0; c < D / 64; ++c) {
-          tma_load_4d(sb + L::OFF_Q + c * L::HALF, &tmQ, bar(L::B_QD), c * 64, hq, i * 128, b);
-          tma_load_4d(sb + L::OFF_DO + c * L::HALF, &tmDO, bar(L::B_QD), c * 64, hq, i * 128, b);
+          tma_load_4d(sb + L::OFF_Q + stg * L::TILE + c * L::HALF, &tmQ, bar(L::B_QD + stg), c * 64,
+                      hq, i * 128, b);
+          tma_load_4d(sb + L::OFF_DO + stg * L::TILE + c * L::HALF, &tmDO, bar(L::B_QD + stg),
+                      c * 64, hq, i * 128, b);
         }
         issued = n + 1;
       }
       // no copy may still be landing at exit
       mbar_wait(bar(L::B_KV), 0, nullptr);
-      if (issued > 0) mbar_wait(bar(L::B_QD), uint32_t((issued - 1) & 1), nullptr);
+      for (int n = max(0, issued - 2); n < issued; ++n)
+        mbar_wait(bar(L::B_QD + (n & 1)), uint32_t((n >> 1) & 1), nullptr);
     }
     __syncwarp();
   }
