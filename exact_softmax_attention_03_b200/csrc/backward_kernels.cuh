@@ -17,15 +17,18 @@
 //                       accumulator with vector atomics
 //   bwd_finalize_kernel dQ accumulator -> bf16
 //
-// bwd_main_kernel warp roles (192 threads):
-//   warps 0-3  elementwise, thread = TMEM lane: first a key row (P, dS), then
-//              a query row (reading dQ); at the end a key row again (dK, dV)
-//   warp 4     tensor-core issuer (whole warp, one elected lane issues)
-//   warp 5     TMA producer (one lane): K_j, V_j once; Q_i, dO_i per block
+// bwd_main_kernel warp roles (320 threads):
+//   warps 0-3  elementwise, thread = TMEM lane = key row: P, dS per block; at
+//              the end dK, dV
+//   warps 4-7  dQ, thread = TMEM lane = query row: read dQ_i out of tensor
+//              memory, add it to the accumulator; stage the next block's
+//              lse2 / delta values in shared memory
+//   warp 8     tensor-core issuer (whole warp, one elected lane issues)
+//   warp 9     TMA producer (one lane): K_j, V_j once; Q_i, dO_i per block
 //              through a 2-stage ring (the next block's tiles load during this one)
 // Per query block (tile = 128 x 128):
-//   Sᵀ  = K_j Q_iᵀ        SS, both K-major                 -> TMEM cols [0,128)
-//   dPᵀ = V_j dO_iᵀ       SS, both K-major                 -> TMEM cols [128,256)
+//   Sᵀ  = K_j Q_iᵀ        SS, both K-major, two 64-query halves -> TMEM cols [0,128)
+//   dPᵀ = V_j dO_iᵀ       SS, both K-major, two 64-query halves -> TMEM cols [128,256)
 //   elementwise: Pᵀ = exp2(Sᵀ c - lse2), dSᵀ = Pᵀ (dPᵀ - delta); Pᵀ and dSᵀ
 //     as bf16 pairs over cols [0,64) and [128,192); dSᵀ also to shared memory
 //   dV += Pᵀ dO_i         TS: A = Pᵀ (TMEM), B = dO_i MN-major
@@ -33,6 +36,10 @@
 //   dQ_i = dS K_j         SS: A = dS MN-major (the dSᵀ tile read transposed),
 //                         B = K_j MN-major; 64 columns of d at a time into the
 //                         free cols [64,128) and [192,256)
+// The first half of the next block's Sᵀ and dPᵀ goes into cols [0,64) and
+// [128,192) as soon as dV and dK are done with them, so the elementwise warps
+// start on it while the dQ warps still read dQ_i out of cols [64,128) and
+// [192,256); the second half follows once that read-out is done.
 // All waits are bounded (sm100_ptx.cuh).
 #pragma once
 
@@ -46,6 +53,45 @@ namespace attn {
 // kind::f16 instruction descriptor with A MN-major too (bit 15).
 __host__ __device__ constexpr uint32_t idesc_bf16_f32_amn(int M, int N, int b_mn_major) {
   return idesc_bf16_f32(M, N, b_mn_major) | (1u << 15);
+}
+
+// 32 lanes x 16 columns of 32-bit from thread i of the warp (lane base + i).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
+        "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]),
+        "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+// Pᵀ and dSᵀ of one key row over 32 queries [c0, c0 + 32) of the block, as
+// bf16 pairs: P = exp2(S c2 - lse2), dS = P (dP - delta). MASK: only the
+// queries in [c_lo, c_hi] are allowed, the rest get P = 0.
+template <bool MASK>
+__device__ __forceinline__ void bwd_p_ds(const uint32_t* sr, const uint32_t* dr, const float* lsr,
+                                         const float* dlt, int c0, int c_lo, int c_hi, float c2,
+                                         uint32_t* pw, uint32_t* dw) {
+  const float4* l4 = reinterpret_cast<const float4*>(lsr + c0);
+  const float4* d4 = reinterpret_cast<const float4*>(dlt + c0);
+#pragma unroll
+  for (int e = 0; e < 32; e += 4) {
+    const float4 lv = l4[e / 4], dv = d4[e / 4];
+    const float l[4] = {lv.x, lv.y, lv.z, lv.w}, d[4] = {dv.x, dv.y, dv.z, dv.w};
+    float pp[4], ds[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float x = fmaf(__uint_as_float(sr[e + u]), c2, -l[u]);
+      pp[u] = ex2_approx(x);
+      if (MASK) pp[u] = (c0 + e + u >= c_lo && c0 + e + u <= c_hi) ? pp[u] : 0.f;
+      ds[u] = pp[u] * (__uint_as_float(dr[e + u]) - d[u]);
+    }
+    pw[e / 2] = pack_bf16x2(pp[0], pp[1]);
+    pw[e / 2 + 1] = pack_bf16x2(pp[2], pp[3]);
+    dw[e / 2] = pack_bf16x2(ds[0], ds[1]);
+    dw[e / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
+  }
 }
 
 struct BwdParams {
@@ -144,24 +190,26 @@ struct BwdLayout {
   static constexpr int B_KV = 0;     // K_j, V_j loaded
   static constexpr int B_QD = 1;     // Q_i, dO_i loaded, + stage
   static constexpr int B_QDE = 3;    // Q_i, dO_i stage free again, + stage
-  static constexpr int B_SD = 5;     // Sᵀ and dPᵀ in TMEM
+  static constexpr int B_SD0 = 5;    // Sᵀ and dPᵀ of queries [0, 64) in TMEM
   static constexpr int B_PR = 6;     // Pᵀ, dSᵀ written (128 arrivals)
   static constexpr int B_QR = 7;     // dQ_i in TMEM
-  static constexpr int B_QF = 8;     // dQ_i read (128 arrivals)
+  static constexpr int B_QF = 8;     // dQ_i read out (128 dQ-warp arrivals)
   static constexpr int B_DONE = 9;   // every dK / dV product complete
-  static constexpr int B_LD = 10;    // per-block lse2 / delta values in shared memory (128 arrivals)
-  static constexpr int NBAR = 11;
+  static constexpr int B_LD = 10;    // block lse2 / delta values in shared memory (128 dQ-warp arrivals)
+  static constexpr int B_SD1 = 11;   // Sᵀ and dPᵀ of queries [64, 128) in TMEM
+  static constexpr int B_KVD = 12;   // dV, dK products of the block complete (issuer only)
+  static constexpr int NBAR = 13;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;      // [0] TMEM base, [1] abort flag
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = BYTES + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_ST = 0, COL_DPT = 128, COL_DV = 256, COL_DK = 256 + D;
-  static constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, 0);
+  static constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64, 0);      // one 64-query half
   static constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, D, 1);
   static constexpr uint32_t IDESC_DQ = idesc_bf16_f32_amn(128, 64, 1);
 };
 
-constexpr int kBwdThreads = 192;
+constexpr int kBwdThreads = 320;
 
 // Query blocks that hold at least one allowed (query, key) pair with a key in
 // [kb0, kb1]: [i_lo, i_hi], empty when i_hi < i_lo.
@@ -215,7 +263,9 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       mbar_init(bar(L::B_QD + st), 1);
       mbar_init(bar(L::B_QDE + st), 1);
     }
-    mbar_init(bar(L::B_SD), 1);
+    mbar_init(bar(L::B_SD0), 1);
+    mbar_init(bar(L::B_SD1), 1);
+    mbar_init(bar(L::B_KVD), 1);
     mbar_init(bar(L::B_PR), 128);
     mbar_init(bar(L::B_QR), 1);
     mbar_init(bar(L::B_QF), 128);
@@ -224,7 +274,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 4) {
+  if (warp == 8) {
     tmem_alloc(smem_u32(tmem_holder), L::TMEM_COLS);
     tmem_relinquish();
   }
@@ -238,31 +288,16 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const int t = int(threadIdx.x);                          // TMEM lane
     const uint32_t lane_off = uint32_t(warp * 32) << 16;
     const uint32_t tST = tmem + lane_off + L::COL_ST, tDPT = tmem + lane_off + L::COL_DPT;
-    // one buffer is enough: block n's values are stored only after B_SD(n),
-    // whose products were issued after every thread arrived on B_QF(n-1),
-    // i.e. after every read of block n-1's values
-    float* lse2_s = reinterpret_cast<float*>(smem + L::OFF_LD);          // [128]
-    float* delta_s = lse2_s + 128;                                       // [128]
+    const float* lsr = reinterpret_cast<const float*>(smem + L::OFF_LD);   // lse2[128]
+    const float* dlt = lsr + 128;                                           // delta[128]
     const int key = kb0 + t;
     const int off = p.Nk - p.Nq;
     const float c2 = p.scale_log2;
     bool ok = true;
     for (int n = 0; ok && n < total; ++n) {
-      const int g = n / nblk, i = i_lo + n % nblk;
-      const int hq = hkv * G + g;
+      const int i = i_lo + n % nblk;
       const int par = n & 1;
-      float l2v, dv;
-      {
-        const int q = i * 128 + t;
-        const bool qv = q < p.Nq;
-        const float l = qv ? __ldg(p.lse + (size_t(b) * p.Hq + hq) * p.Nq + q) : 0.f;
-        l2v = (qv && l > -CUDART_INF_F) ? l * 1.4426950408889634f : 0.f;
-        dv = qv ? __ldg(p.delta + (size_t(b) * p.Hq + hq) * p.Nq + q) : 0.f;
-      }
-      if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_SD), uint32_t(par), abort_flag)))) break;
-      lse2_s[t] = l2v;
-      delta_s[t] = dv;
-      mbar_arrive(bar(L::B_LD));
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_SD0), uint32_t(par), abort_flag)))) break;
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_LD), uint32_t(par), abort_flag)))) break;
       tc_fence_after();
       // allowed queries of this key within the block: [c_lo, c_hi]
@@ -271,75 +306,42 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       if (key >= p.Nk) c_hi = -1;
       if (p.causal) c_lo = max(c_lo, key - off - q0);                    // key <= q + off
       if (p.window_left >= 0) c_hi = min(c_hi, key + p.window_left - off - q0);
-      const float* lsr = lse2_s;
-      const float* dlt = delta_s;
-      // 64 queries at a time: read their Sᵀ and dPᵀ columns (32 at a time),
-      // then write the bf16 pairs of Pᵀ and dSᵀ over columns already read
+      // 32 queries at a time: read their Sᵀ and dPᵀ columns, then write the
+      // bf16 pairs of Pᵀ and dSᵀ over columns already read (chunk c of 32
+      // queries -> columns [16c, 16c + 16))
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t pw[32], dw[32];
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          const int c0 = 64 * h + 32 * cc;
-          uint32_t sr[32], dr[32];
-          tmem_ld32(tST + c0, sr);
-          tmem_ld32(tDPT + c0, dr);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            float pp[2], ds[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int c = c0 + e + u;
-              const bool al = c >= c_lo && c <= c_hi;
-              const float x = fmaf(__uint_as_float(sr[e + u]), c2, -lsr[c]);
-              pp[u] = al ? ex2_approx(x) : 0.f;
-              ds[u] = pp[u] * (__uint_as_float(dr[e + u]) - dlt[c]);
-            }
-            pw[16 * cc + e / 2] = pack_bf16x2(pp[0], pp[1]);
-            dw[16 * cc + e / 2] = pack_bf16x2(ds[0], ds[1]);
-          }
+      for (int cc = 0; cc < 4; ++cc) {
+        const int c0 = 32 * cc;
+        if (cc == 2) {                                       // second 64-query half
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_SD1), uint32_t(par), abort_flag)))) break;
+          tc_fence_after();
         }
-        tmem_st32(tST + 32 * h, pw);
-        tmem_st32(tDPT + 32 * h, dw);
-        // dSᵀ row of this key -> shared memory block h (queries 64h..64h+63),
+        uint32_t sr[32], dr[32], pw[16], dw[16];
+        tmem_ld32(tST + c0, sr);
+        tmem_ld32(tDPT + c0, dr);
+        tmem_wait_ld();
+        if (__all_sync(0xffffffffu, c_lo <= c0 && c_hi >= c0 + 31))
+          bwd_p_ds<false>(sr, dr, lsr, dlt, c0, c_lo, c_hi, c2, pw, dw);
+        else
+          bwd_p_ds<true>(sr, dr, lsr, dlt, c0, c_lo, c_hi, c2, pw, dw);
+        tmem_st16(tST + 16 * cc, pw);
+        tmem_st16(tDPT + 16 * cc, dw);
+        // dSᵀ row of this key -> shared memory block cc / 2 (queries 64h..64h+63),
         // 16-byte chunks swizzled by (row & 7)
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          const uint32_t addr = sb + L::OFF_DS + h * L::HALF + t * 128 + ((ch ^ (t & 7)) * 16);
+        for (int ch = 0; ch < 4; ++ch) {
+          const int chunk = 4 * (cc & 1) + ch;
+          const uint32_t addr = sb + L::OFF_DS + (cc >> 1) * L::HALF + t * 128 + ((chunk ^ (t & 7)) * 16);
           asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
                        ::"r"(addr), "r"(dw[4 * ch]), "r"(dw[4 * ch + 1]), "r"(dw[4 * ch + 2]),
                        "r"(dw[4 * ch + 3]) : "memory");
         }
       }
+      if (!ok) break;
       tmem_wait_st();
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       tc_fence_before();
       mbar_arrive(bar(L::B_PR));
-      // ---- dQ rows: thread t is now query row q0 + t ----------------------
-      if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_QR), uint32_t(par), abort_flag)))) break;
-      tc_fence_after();
-      uint32_t qr[D];
-#pragma unroll
-      for (int h = 0; h < D / 64; ++h) {
-        const uint32_t col = (h == 0 ? tST : tDPT) + 64;
-        tmem_ld32(col, qr + 64 * h);
-        tmem_ld32(col + 32, qr + 64 * h + 32);
-      }
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bar(L::B_QF));
-      const int q = q0 + t;
-      if (q < p.Nq) {
-        // chunk e of query q: the warp's 32 queries are 32 adjacent float4
-        float4* dst = reinterpret_cast<float4*>(p.dq_acc) + (size_t(b) * p.Hq + hq) * (D / 4) * p.Nq + q;
-#pragma unroll
-        for (int e = 0; e < D / 4; ++e)
-          atomicAdd(dst + size_t(e) * p.Nq, make_float4(__uint_as_float(qr[4 * e]) * p.scale,
-                                         __uint_as_float(qr[4 * e + 1]) * p.scale,
-                                         __uint_as_float(qr[4 * e + 2]) * p.scale,
-                                         __uint_as_float(qr[4 * e + 3]) * p.scale));
-      }
     }
     // ---- dK, dV of this key row ---------------------------------------------
     const bool have = ok && total > 0 &&
@@ -375,7 +377,63 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         }
       }
     }
-  } else if (warp == 4) {
+  } else if (warp < 8) {
+    // ======================= dQ warps ========================================
+    const int r = int(threadIdx.x) - 128;                    // TMEM lane = query row in the block
+    const uint32_t lane_off = uint32_t((warp - 4) * 32) << 16;
+    float* lse2_s = reinterpret_cast<float*>(smem + L::OFF_LD);
+    float* delta_s = lse2_s + 128;
+    // lse2 (log2 units, 0 for empty rows) and delta of query row r of block n
+    auto row_values = [&](int n, float& l2, float& dl) {
+      const int hq = hkv * G + n / nblk, q = (i_lo + n % nblk) * 128 + r;
+      const bool qv = q < p.Nq;
+      const float l = qv ? __ldg(p.lse + (size_t(b) * p.Hq + hq) * p.Nq + q) : 0.f;
+      l2 = (qv && l > -CUDART_INF_F) ? l * 1.4426950408889634f : 0.f;
+      dl = qv ? __ldg(p.delta + (size_t(b) * p.Hq + hq) * p.Nq + q) : 0.f;
+    };
+    if (total > 0) {
+      float l2, dl;
+      row_values(0, l2, dl);
+      lse2_s[r] = l2;
+      delta_s[r] = dl;
+      mbar_arrive(bar(L::B_LD));
+    }
+    for (int n = 0; n < total; ++n) {
+      const int hq = hkv * G + n / nblk, q = (i_lo + n % nblk) * 128 + r;
+      float l2 = 0.f, dl = 0.f;
+      if (n + 1 < total) row_values(n + 1, l2, dl);
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_QR), uint32_t(n & 1), abort_flag))) break;
+      tc_fence_after();
+      // one buffer is enough: B_QR(n) completes after the products issued once
+      // every elementwise thread arrived on B_PR(n), i.e. after every read of
+      // block n's values
+      if (n + 1 < total) {
+        lse2_s[r] = l2;
+        delta_s[r] = dl;
+        mbar_arrive(bar(L::B_LD));
+      }
+      uint32_t qr[D];
+#pragma unroll
+      for (int h = 0; h < D / 64; ++h) {
+        const uint32_t col = tmem + lane_off + (h == 0 ? L::COL_ST : L::COL_DPT) + 64;
+        tmem_ld32(col, qr + 64 * h);
+        tmem_ld32(col + 32, qr + 64 * h + 32);
+      }
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar(L::B_QF));
+      if (q < p.Nq) {
+        // chunk e of query q: the warp's 32 queries are 32 adjacent float4
+        float4* dst = reinterpret_cast<float4*>(p.dq_acc) + (size_t(b) * p.Hq + hq) * (D / 4) * p.Nq + q;
+#pragma unroll
+        for (int e = 0; e < D / 4; ++e)
+          atomicAdd(dst + size_t(e) * p.Nq, make_float4(__uint_as_float(qr[4 * e]) * p.scale,
+                                                        __uint_as_float(qr[4 * e + 1]) * p.scale,
+                                                        __uint_as_float(qr[4 * e + 2]) * p.scale,
+                                                        __uint_as_float(qr[4 * e + 3]) * p.scale));
+      }
+    }
+  } else if (warp == 8) {
     // ======================= tensor-core issuer ==============================
     auto wwait = [&](int bi, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(bar(bi), parity, abort_flag));
@@ -392,26 +450,36 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const uint64_t dKj_mn = smem_desc_sw128(sb + L::OFF_K, L::HALF, 1024);
     const uint32_t tST = tmem + L::COL_ST, tDPT = tmem + L::COL_DPT;
     const uint32_t tDV = tmem + L::COL_DV, tDK = tmem + L::COL_DK;
-    bool alive = total > 0 && wwait(L::B_KV, 0u);
+    // Sᵀ = K_j Q_iᵀ and dPᵀ = V_j dO_iᵀ (K = d) for queries [64h, 64h + 64) of
+    // block n: TMEM cols [64h, 64h + 64) of each
+    auto issue_sdp = [&](int n, int h) {
+      const uint32_t so = uint32_t(((n & 1) * L::TILE + h * 64 * 128) >> 4);
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t o = ((k / 4) * L::HALF + (k % 4) * 32) >> 4;
+        if (elect_one()) mma_ss(tST + 64 * h, dK_k + o, dQ_k + so + o, L::IDESC_S, k > 0 ? 1u : 0u);
+      }
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t o = ((k / 4) * L::HALF + (k % 4) * 32) >> 4;
+        if (elect_one()) mma_ss(tDPT + 64 * h, dV_k + o, dO_k + so + o, L::IDESC_S, k > 0 ? 1u : 0u);
+      }
+    };
+    bool alive = total > 0 && wwait(L::B_KV, 0u) && wwait(L::B_QD, 0u);
+    if (alive) {
+      tc_fence_after();
+      issue_sdp(0, 0);
+      commit(L::B_SD0);
+    }
     for (int n = 0; alive && n < total; ++n) {
       const uint32_t par = uint32_t(n & 1);
       const int stg = n & 1;                                     // Q/dO stage of this block
       const uint32_t so = uint32_t(stg * (L::TILE >> 4));       // its descriptor offset
-      if (!(alive = wwait(L::B_QD + stg, uint32_t((n >> 1) & 1)))) break;
-      if (n > 0 && !(alive = wwait(L::B_QF, par ^ 1u))) break;   // previous dQ read out
+      // second half once dQ of the previous block (cols [64, 128)) is read out
+      if (n > 0 && !(alive = wwait(L::B_QF, par ^ 1u))) break;
       tc_fence_after();
-      // Sᵀ = K_j Q_iᵀ and dPᵀ = V_j dO_iᵀ (K = d)
-#pragma unroll
-      for (int k = 0; k < D / 16; ++k) {
-        const uint32_t o = ((k / 4) * L::HALF + (k % 4) * 32) >> 4;
-        if (elect_one()) mma_ss(tST, dK_k + o, dQ_k + so + o, L::IDESC_S, k > 0 ? 1u : 0u);
-      }
-#pragma unroll
-      for (int k = 0; k < D / 16; ++k) {
-        const uint32_t o = ((k / 4) * L::HALF + (k % 4) * 32) >> 4;
-        if (elect_one()) mma_ss(tDPT, dV_k + o, dO_k + so + o, L::IDESC_S, k > 0 ? 1u : 0u);
-      }
-      commit(L::B_SD);
+      issue_sdp(n, 1);
+      commit(L::B_SD1);
       if (!(alive = wwait(L::B_PR, par))) break;
       tc_fence_after();
       // dV += Pᵀ dO_i, dK += dSᵀ Q_i (K = 128 queries, 16 per MMA)
@@ -425,6 +493,8 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const uint32_t o = (k * 16 * 128) >> 4;
         if (elect_one()) mma_ts(tDK, tDPT + 8 * k, dQ_mn + so + o, L::IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
       }
+      const bool next = n + 1 < total;
+      if (next) commit(L::B_KVD);
       // dQ_i = dS K_j, 64 columns of d at a time (K = 128 keys)
 #pragma unroll
       for (int h = 0; h < D / 64; ++h) {
@@ -438,13 +508,22 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
       commit(L::B_QR);
       commit(L::B_QDE + stg);
+      if (next) {
+        // first half of the next block: its columns [0, 64) held Pᵀ and dSᵀ,
+        // free once the dV and dK products finished reading them
+        if (!(alive = wwait(L::B_QD + ((n + 1) & 1), uint32_t(((n + 1) >> 1) & 1)))) break;
+        if (!(alive = wwait(L::B_KVD, par))) break;
+        tc_fence_after();
+        issue_sdp(n + 1, 0);
+        commit(L::B_SD0);
+      }
     }
     if (total > 0) {
       commit(L::B_DONE);                        // also drains every issued product
       mbar_wait(bar(L::B_DONE), 0, nullptr);
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ======================= TMA producer ====================================
     if (lane == 0 && total > 0) {
       tma_prefetch_desc(&tmQ);
@@ -482,7 +561,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == 8) {
     tc_fence_after();
     tmem_dealloc(tmem, L::TMEM_COLS);
   }
