@@ -53,3 +53,19 @@ def sample_rows(n, k, seed):
     g = torch.Generator().manual_seed(seed)
     pick = torch.randperm(n, generator=g)[:max(0, k - 2)].tolist()
     return sorted(set(pick) | {0, n - 1})
+
+
+def backward_of_group(q, k, v, dout, b, hk, causal, window_left):
+    """Oracle dQ, dK, dV of one (batch, K/V head) and its group of query heads.
+
+    The gradients of a K/V head and the dQ of its query heads depend only on
+    that group's inputs, so a full-size problem can be checked one group at a
+    time. Returns (dQ [Nq, G, d], dK [Nk, d], dV [Nk, d]) in fp64.
+    """
+    import oracle
+    G = q.shape[2] // k.shape[2]
+    hs = slice(hk * G, (hk + 1) * G)
+    dq, dk, dv = oracle.oracle_attention_backward(
+        q[b:b + 1, :, hs], k[b:b + 1, :, hk:hk + 1], v[b:b + 1, :, hk:hk + 1],
+        dout[b:b + 1, :, hs], causal=causal, window_left=window_left)
+    return dq[0], dk[0, :, 0], dv[0, :, 0]

@@ -82,3 +82,22 @@ def test_masked_rows_give_zero_query_gradient():
     do = rng.standard_normal((1, 6, 1, 4))
     dQ, _, _ = oracle.oracle_attention_backward(q, k, v, do, causal=True)
     assert np.all(dQ[0, :3] == 0)           # rows 0-2 see no key (bottom-right alignment)
+
+
+def test_group_slices_equal_the_full_problem():
+    # the full-size GPU parity test checks one (batch, K/V head) group at a time
+    from parity import backward_of_group
+    rng = np.random.default_rng(5)
+    B, Hq, Hkv, Nq, Nk, d = 2, 6, 2, 9, 13, 4
+    q = rng.standard_normal((B, Nq, Hq, d))
+    k = rng.standard_normal((B, Nk, Hkv, d))
+    v = rng.standard_normal((B, Nk, Hkv, d))
+    do = rng.standard_normal((B, Nq, Hq, d))
+    dQ, dK, dV = oracle.oracle_attention_backward(q, k, v, do, causal=True, window_left=5)
+    G = Hq // Hkv
+    for b in range(B):
+        for hk in range(Hkv):
+            gq, gk, gv = backward_of_group(q, k, v, do, b, hk, True, 5)
+            assert np.allclose(gq, dQ[b, :, hk * G:(hk + 1) * G], rtol=0, atol=1e-12)
+            assert np.allclose(gk, dK[b, :, hk], rtol=0, atol=1e-12)
+            assert np.allclose(gv, dV[b, :, hk], rtol=0, atol=1e-12)

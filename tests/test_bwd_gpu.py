@@ -14,7 +14,7 @@ import torch
 
 import attn_inputs as ai
 import oracle
-from parity import cuda
+from parity import backward_of_group, cuda
 
 pytestmark = pytest.mark.gpu
 
@@ -30,7 +30,8 @@ def _built():
     build.build()
 
 
-def run_bwd(B, Hq, Hkv, Nq, Nk, d, causal, wl):
+def gpu_bwd(B, Hq, Hkv, Nq, Nk, d, causal, wl):
+    """Inputs (CPU, bf16) and the GPU gradients, with O and LSE from attn_fwd."""
     import exact_softmax_attention_03_b200 as ea
     q, k, v = ai.make_qkv(B, Hq, Hkv, Nq, Nk, d)
     do = ai.make_dout(B, Nq, Hq, d)
@@ -39,12 +40,17 @@ def run_bwd(B, Hq, Hkv, Nq, Nk, d, causal, wl):
     o, _ = ea.attn_fwd(qg, kg, vg, lse=lse, causal=causal, window_left=wl)
     dq, dk, dv = ea.attn_bwd(qg, kg, vg, o, lse, dog, causal=causal, window_left=wl)
     assert ea.attn_device_status() == 0
+    return (q, k, v, do), (dq, dk, dv)
+
+
+def run_bwd(B, Hq, Hkv, Nq, Nk, d, causal, wl):
+    (q, k, v, do), got = gpu_bwd(B, Hq, Hkv, Nq, Nk, d, causal, wl)
     ref = oracle.oracle_attention_backward(q, k, v, do, causal=causal, window_left=wl)
-    return (dq, dk, dv), ref
+    return got, ref
 
 
-def check(shape, causal, wl):
-    got, ref = run_bwd(*shape, causal, wl)
+def compare(got, ref, what):
+    """rel-L2 and largest error relative to the largest reference magnitude."""
     errs = {}
     for name, g, r in zip(("dq", "dk", "dv"), got, ref):
         g = g.float().cpu().numpy().astype(np.float64)
@@ -53,11 +59,16 @@ def check(shape, causal, wl):
         e = {"rel_l2": float(np.linalg.norm(g - r) / max(np.linalg.norm(r), 1e-30)),
              "max_rel": float(np.abs(g - r).max() / scale)}
         errs[name] = e
-        print(shape, causal, wl, name, e)
+        print(what, name, e)
     for name, e in errs.items():
-        assert e["rel_l2"] <= REL_L2[name], (shape, causal, wl, name, errs)
-        assert e["max_rel"] <= MAX_REL, (shape, causal, wl, name, errs)
+        assert e["rel_l2"] <= REL_L2[name], (what, name, errs)
+        assert e["max_rel"] <= MAX_REL, (what, name, errs)
     return errs
+
+
+def check(shape, causal, wl):
+    got, ref = run_bwd(*shape, causal, wl)
+    return compare(got, ref, (shape, causal, wl))
 
 
 SHAPES = [
@@ -82,3 +93,27 @@ def test_rows_without_keys_get_zero_query_gradient():
     got, _ = run_bwd(1, 2, 2, 300, 100, 128, True, -1)
     dq = got[0]
     assert (dq[:, :200].float() == 0).all()
+
+
+FULL = [
+    # the backward workload the bench times (MHA causal B4 H32 N2048 d128), and a
+    # GQA windowed problem of the same size; same launch configuration
+    ((4, 32, 32, 2048, 2048, 128), True, -1),
+    ((2, 32, 8, 2048, 2048, 128), True, 512),
+]
+
+
+@pytest.mark.parametrize("shape,causal,wl", FULL)
+def test_full_size_sampled_groups(shape, causal, wl):
+    B, Hq, Hkv, Nq, Nk, d = shape
+    G = Hq // Hkv
+    (q, k, v, do), (dq, dk, dv) = gpu_bwd(*shape, causal, wl)
+    for t in (dq, dk, dv):
+        assert torch.isfinite(t.float()).all()
+    g = torch.Generator().manual_seed(7)
+    picks = [(0, 0), (B - 1, Hkv - 1),
+             (int(torch.randint(B, (1,), generator=g)), int(torch.randint(Hkv, (1,), generator=g)))]
+    for b, hk in picks:
+        ref = backward_of_group(q, k, v, do, b, hk, causal, wl)
+        got = (dq[b, :, hk * G:(hk + 1) * G], dk[b, :, hk], dv[b, :, hk])
+        compare(got, ref, (shape, causal, wl, b, hk))
