@@ -50,6 +50,8 @@ KERNEL_SOURCES = {
                for f in ("sm100_ptx.cuh", "decode_kernels.cuh")],
     "decode_paged": ["exact_softmax_attention_03_b200/csrc/" + f
                      for f in ("sm100_ptx.cuh", "decode_kernels.cuh")],
+    "bwd_main_kernel": ["exact_softmax_attention_03_b200/csrc/" + f
+                        for f in ("sm100_ptx.cuh", "backward_kernels.cuh")],
 }
 
 
@@ -94,10 +96,14 @@ def kernel_source_hash(kernel: str) -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from a committed ncu summary, if taken on these sources."""
+def recorded_traffic(kernel: str, workload: str, resized: bool = False):
+    """DRAM bytes per launch from a committed ncu summary, if taken on these sources.
+
+    The recorded figures are per launch of the full workload: none is reported
+    when the run overrides the workload's batch (``resized``).
+    """
     path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
-    if not os.path.exists(path):
+    if resized or not os.path.exists(path):
         return None
     want = kernel_source_hash(kernel)
     with open(path) as f:
@@ -538,7 +544,7 @@ def run_ours(args, world, rank, local):
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
                      "frac": achieved / peak_t, "peak_source": f"{peak_src} bf16_tflops (burst)",
                      "kernel": "attn_fwd_kernel<128,false>",
-                     "traffic": recorded_traffic("attn_fwd_kernel", args.workload),
+                     "traffic": recorded_traffic("attn_fwd_kernel", args.workload, bool(args.batch)),
                      "algorithmic_bytes": metrics.attn_fwd_bytes(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d)},
         "decode": {
             "workload": dw.name, "value": d_value, "unit": "GB/s", "ms_per_step": dms_max,
@@ -548,7 +554,7 @@ def run_ours(args, world, rank, local):
                          "peak_source": f"{peak_src} hbm_gbs",
                          "kernel": "decode_split_kernel<128,4> + decode_combine_kernel<128>",
                          "algorithmic_bytes": d_all,
-                         "traffic": recorded_traffic("decode", "decode")},
+                         "traffic": recorded_traffic("decode", "decode", bool(args.decode_batch))},
             "gpu_launches": dlaunches,
         },
         "backward": {
@@ -559,7 +565,8 @@ def run_ours(args, world, rank, local):
                          "unit": "TFLOP/s", "frac": b_achieved / peak_t,
                          "peak_source": f"{peak_src} bf16_tflops (burst)",
                          "kernel": "bwd_prep_kernel + bwd_main_kernel<128> + bwd_finalize_kernel",
-                         "traffic": None},
+                         "traffic": recorded_traffic("bwd_main_kernel", args.workload, bool(args.batch)),
+                         "traffic_kernel": "bwd_main_kernel<128>"},
             "gpu_launches": blaunches,
         },
         "merge": {
@@ -591,7 +598,7 @@ def run_ours(args, world, rank, local):
                          "peak_source": f"{peak_src} hbm_gbs",
                          "kernel": "decode_split_kernel<128,4,paged> + decode_combine_kernel<128>",
                          "algorithmic_bytes": d_all,
-                         "traffic": recorded_traffic("decode_paged", f"decode_p{ps}")},
+                         "traffic": recorded_traffic("decode_paged", f"decode_p{ps}", bool(args.decode_batch))},
             "gpu_launches": plaunches,
         },
         "clocks": clocks,
