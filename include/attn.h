@@ -58,7 +58,7 @@ typedef enum {
   ATTN_ERR_UNSUPPORTED = 2,   /* device is not sm_100, or head dim not in {64, 128} */
   ATTN_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed (message has the code) */
   ATTN_ERR_TIMEOUT = 4,       /* a bounded device-side wait gave up (see attn_device_status) */
-  ATTN_ERR_WORKSPACE = 5      /* decode workspace missing or smaller than required */
+  ATTN_ERR_WORKSPACE = 5      /* decode or backward workspace missing or smaller than required */
 } attn_status;
 
 /*
