@@ -113,6 +113,9 @@ int make_map(CUtensorMap* map, const void* base, int d, int H, int N, int B, int
 bool finite_pos(float x) { return std::isfinite(x) && x > 0.f; }
 
 constexpr long long kMaxIndex = (1ll << 31) - 1;
+// longest cache a decode call takes: its split length, rounded up to whole
+// 128-key tiles, must still fit the kernels' 32-bit positions
+constexpr long long kMaxKeys = kMaxIndex - 127;
 
 int validate_fwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
                  int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal) {
@@ -260,7 +263,7 @@ int decode_group_tile(int G) {
 // items round-robin), each item streaming at least one 128-key tile.
 int auto_splits(int B, int Hq, int Lmax) {
   const long long base = std::max(1ll, (static_cast<long long>(B) * Hq + 3) / 4);
-  const int cap = std::max(1, std::min(64, (Lmax + 127) / 128));
+  const int cap = static_cast<int>(std::max(1ll, std::min(64ll, (static_cast<long long>(Lmax) + 127) / 128)));
   int best = cap;
   for (int s = 1; s <= cap; ++s) {
     const long long items = base * s;
@@ -274,21 +277,28 @@ struct DecodeShape {
   int S;
   int chunk;
   size_t acc_bytes, ml_bytes, total;
+  bool too_large;     // the workspace would exceed 2^62 bytes
 };
 
 DecodeShape decode_shape(int B, int Hq, int d, int num_splits, int Lmax) {
+  // callers pass 1 <= Lmax <= kMaxKeys; 64-bit so that no sum below overflows
   DecodeShape s{};
-  int S = num_splits > 0 ? num_splits : auto_splits(B, Hq, Lmax);
-  if (S > Lmax) S = Lmax;
-  const int quantum = 128;                          // keys per K/V tile
-  int chunk = (Lmax + S - 1) / S;
+  const long long L = Lmax;
+  long long S = num_splits > 0 ? num_splits : auto_splits(B, Hq, Lmax);
+  if (S > L) S = L;
+  const long long quantum = 128;                    // keys per K/V tile
+  long long chunk = (L + S - 1) / S;
   chunk = (chunk + quantum - 1) / quantum * quantum;
-  S = (Lmax + chunk - 1) / chunk;
-  s.S = S;
-  s.chunk = chunk;
+  S = (L + chunk - 1) / chunk;
+  s.S = static_cast<int>(S);
+  s.chunk = static_cast<int>(chunk);
+  // B * Hq * S * (d + 2) floats can pass 2^64 for extreme sizes: count in 128 bits
+  const unsigned __int128 rows = static_cast<unsigned __int128>(B) * Hq * S;
+  s.too_large = rows * (d + 2) * sizeof(float) > (static_cast<unsigned __int128>(1) << 62);
+  if (s.too_large) return s;
   auto round256 = [](size_t x) { return (x + 255) / 256 * 256; };
-  s.acc_bytes = round256(static_cast<size_t>(B) * Hq * S * d * sizeof(float));
-  s.ml_bytes = round256(static_cast<size_t>(B) * Hq * S * 2 * sizeof(float));
+  s.acc_bytes = round256(static_cast<size_t>(rows) * d * sizeof(float));
+  s.ml_bytes = round256(static_cast<size_t>(rows) * 2 * sizeof(float));
   s.total = s.acc_bytes + s.ml_bytes;
   return s;
 }
@@ -323,8 +333,8 @@ int launch_decode_kernels(attn::DecodeParams& p, const void* k_cache, const void
   }
   const int grid = static_cast<int>(std::min<long long>(items, sms));
   attn::decode_split_kernel<D, GT, PAGED><<<grid, attn::kDecodeSplitThreads, L::SMEM_ALLOC, stream>>>(mk, mv, p);
-  const int n = p.B * p.Hq;
-  attn::decode_combine_kernel<D><<<(n + 3) / 4, 128, 0, stream>>>(p);
+  const long long n = static_cast<long long>(p.B) * p.Hq;
+  attn::decode_combine_kernel<D><<<unsigned((n + 3) / 4), 128, 0, stream>>>(p);
   return ATTN_OK;
 }
 
@@ -430,9 +440,11 @@ int attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
     return fail(ATTN_ERR_INVALID_ARG, "q, k_cache, v_cache, o must be 16-byte aligned");
   if (lse && !aligned(lse, 4)) return fail(ATTN_ERR_INVALID_ARG, "lse must be 4-byte aligned");
   if (seqlens && !aligned(seqlens, 4)) return fail(ATTN_ERR_INVALID_ARG, "seqlens must be 4-byte aligned");
-  if (static_cast<long long>(B) * Lmax > kMaxIndex || static_cast<long long>(B) * Hq > kMaxIndex)
+  if (static_cast<long long>(B) * Lmax > kMaxIndex || static_cast<long long>(B) * Hq > kMaxIndex ||
+      Lmax > kMaxKeys)
     return fail(ATTN_ERR_INVALID_ARG, "sizes too large");
   const DecodeShape sh = decode_shape(B, Hq, d, num_splits, Lmax);
+  if (sh.too_large) return fail(ATTN_ERR_INVALID_ARG, "sizes too large");
   if (sh.total > ATTN_DECODE_NOALLOC_SCRATCH_BYTES)
     return fail(ATTN_ERR_WORKSPACE,
                 "these sizes need %zu bytes of scratch (%d splits) but the fixed scratch holds %zu; "
@@ -500,6 +512,10 @@ int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float*
 
 size_t attn_bwd_workspace_bytes(int B, int Hq, int Nq, int d) {
   if (B < 1 || Hq < 1 || Nq < 1 || (d != 64 && d != 128)) return 0;
+  // the size limits attn_bwd applies
+  if (static_cast<long long>(B) * Nq > kMaxIndex || static_cast<long long>(B) * Hq > kMaxIndex ||
+      static_cast<long long>(B) * Nq * Hq > kMaxIndex * 8ll / d)
+    return 0;
   return bwd_ws_bytes(B, Hq, Nq, d);
 }
 
@@ -513,7 +529,8 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const v
     return fail(ATTN_ERR_INVALID_ARG, "dout, lse, dq, dk and dv must be non-null");
   if (!aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16))
     return fail(ATTN_ERR_INVALID_ARG, "dout, dq, dk, dv must be 16-byte aligned");
-  if (static_cast<long long>(B) * Nq * Hq * d > kMaxIndex * 8ll)
+  // B * Nq and B * Hq are below 2^31 here, so B * Nq * Hq fits 64 bits
+  if (static_cast<long long>(B) * Nq * Hq > kMaxIndex * 8ll / d)
     return fail(ATTN_ERR_INVALID_ARG, "sizes too large");
   const size_t need = bwd_ws_bytes(B, Hq, Nq, d);
   if (workspace == nullptr || workspace_bytes < need)
@@ -554,8 +571,10 @@ int attn_merge(const float* o_parts, const float* lse_parts, int R, void* o, flo
   if (d != 64 && d != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim %d not in {64, 128}", d);
   if (!aligned(o_parts, 16) || !aligned(o, 8) || !aligned(lse_parts, 4) || (lse && !aligned(lse, 4)))
     return fail(ATTN_ERR_INVALID_ARG, "o_parts must be 16-byte, o 8-byte, lse 4-byte aligned");
-  const long long rows = static_cast<long long>(B) * Nq * Hq;
-  if (rows * d > kMaxIndex * 16ll || rows * R > kMaxIndex * 16ll)
+  if (static_cast<long long>(B) * Nq > kMaxIndex || static_cast<long long>(B) * Hq > kMaxIndex)
+    return fail(ATTN_ERR_INVALID_ARG, "sizes too large");
+  const long long rows = static_cast<long long>(B) * Nq * Hq;     // < 2^62 here
+  if (rows > kMaxIndex * 16ll / d || rows > kMaxIndex * 16ll / R)
     return fail(ATTN_ERR_INVALID_ARG, "sizes too large");
   int dev = 0;
   int rc = check_device(&dev);
@@ -585,8 +604,10 @@ int attn_merge(const float* o_parts, const float* lse_parts, int R, void* o, flo
 }
 
 size_t attn_decode_workspace_bytes(int B, int Hq, int d, int num_splits, int Lmax) {
-  if (B < 1 || Hq < 1 || Lmax < 1 || (d != 64 && d != 128) || num_splits < 0) return 0;
-  return decode_shape(B, Hq, d, num_splits, Lmax).total;
+  if (B < 1 || Hq < 1 || Lmax < 1 || Lmax > kMaxKeys || (d != 64 && d != 128) || num_splits < 0)
+    return 0;
+  const DecodeShape sh = decode_shape(B, Hq, d, num_splits, Lmax);
+  return sh.too_large ? 0 : sh.total;
 }
 
 int attn_decode(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
@@ -605,9 +626,11 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache, void* o
     return fail(ATTN_ERR_INVALID_ARG, "q, k_cache, v_cache, o must be 16-byte aligned");
   if (lse && !aligned(lse, 4)) return fail(ATTN_ERR_INVALID_ARG, "lse must be 4-byte aligned");
   if (seqlens && !aligned(seqlens, 4)) return fail(ATTN_ERR_INVALID_ARG, "seqlens must be 4-byte aligned");
-  if (static_cast<long long>(B) * Lmax > kMaxIndex || static_cast<long long>(B) * Hq > kMaxIndex)
+  if (static_cast<long long>(B) * Lmax > kMaxIndex || static_cast<long long>(B) * Hq > kMaxIndex ||
+      Lmax > kMaxKeys)
     return fail(ATTN_ERR_INVALID_ARG, "sizes too large");
   const DecodeShape sh = decode_shape(B, Hq, d, num_splits, Lmax);
+  if (sh.too_large) return fail(ATTN_ERR_INVALID_ARG, "sizes too large");
   if (workspace == nullptr || workspace_bytes < sh.total)
     return fail(ATTN_ERR_WORKSPACE, "workspace of %zu bytes needed, got %zu", sh.total,
                 workspace == nullptr ? size_t(0) : workspace_bytes);
@@ -659,10 +682,11 @@ int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, v
   if (lse && !aligned(lse, 4)) return fail(ATTN_ERR_INVALID_ARG, "lse must be 4-byte aligned");
   if (seqlens && !aligned(seqlens, 4)) return fail(ATTN_ERR_INVALID_ARG, "seqlens must be 4-byte aligned");
   const long long Lmax = static_cast<long long>(pages_per_seq) * page_size;
-  if (Lmax > kMaxIndex || static_cast<long long>(B) * pages_per_seq > kMaxIndex ||
+  if (Lmax > kMaxKeys || static_cast<long long>(B) * pages_per_seq > kMaxIndex ||
       static_cast<long long>(B) * Hq > kMaxIndex || static_cast<long long>(num_pages) >= kMaxIndex)
     return fail(ATTN_ERR_INVALID_ARG, "sizes too large");
   const DecodeShape sh = decode_shape(B, Hq, d, num_splits, static_cast<int>(Lmax));
+  if (sh.too_large) return fail(ATTN_ERR_INVALID_ARG, "sizes too large");
   if (workspace == nullptr || workspace_bytes < sh.total)
     return fail(ATTN_ERR_WORKSPACE, "workspace of %zu bytes needed, got %zu", sh.total,
                 workspace == nullptr ? size_t(0) : workspace_bytes);
