@@ -39,6 +39,12 @@
  * Errors. Every entry point validates its arguments on the host first; on any
  * error it returns a non-zero attn_status, launches nothing, and records a
  * message readable with attn_last_error() (thread-local).
+ *
+ * Size limits (ATTN_ERR_INVALID_ARG beyond them): the kernels index rows and
+ * positions in 32 bits, so B * Nq, B * Nk, B * Hq (and B * Lmax for decode)
+ * stay below 2^31; a decode cache holds at most 2^31 - 128 keys; the backward
+ * pass needs B * Nq * Hq * d <= 8 * (2^31 - 1); a decode workspace may not
+ * exceed 2^62 bytes.
  */
 #ifndef ATTN_H_
 #define ATTN_H_
@@ -124,6 +130,8 @@ int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float*
  *          256-byte aligned (fp32 dQ accumulator and per-row dO.O sums)
  *   other arguments : as attn_fwd (the same causal / window_left / scale)
  * Returns ATTN_OK or an attn_status; nothing is launched on error.
+ * attn_bwd_workspace_bytes returns 0 for invalid sizes or sizes past the
+ * limits above.
  */
 size_t attn_bwd_workspace_bytes(int B, int Hq, int Nq, int d);
 int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
@@ -152,7 +160,7 @@ int attn_merge(const float* o_parts, const float* lse_parts, int R, void* o, flo
 /*
  * Bytes of device workspace attn_decode needs for these sizes.
  * num_splits = 0 picks the split count attn_decode would pick automatically.
- * Returns 0 for invalid sizes.
+ * Returns 0 for invalid sizes, including sizes past the limits above.
  */
 size_t attn_decode_workspace_bytes(int B, int Hq, int d, int num_splits, int Lmax);
 
