@@ -15,6 +15,11 @@ Causal masking across chunks: rank r's queries sit at global positions
 (diagonal) block, chunks s > r are wholly masked and skipped. Sliding windows
 are not supported here. All arithmetic runs in the library's kernels; this
 module only moves tensors and chooses calls.
+
+Two ways to reach the other ranks' chunks: ``context_parallel_attention``
+all-gathers them (NCCL), ``context_parallel_attention_peer`` lets the forward
+kernel read them in place from the owners' memory (``PeerKV``), so the
+transfer overlaps the products tile by tile and no gathered copy is made.
 """
 
 from __future__ import annotations
@@ -67,3 +72,62 @@ def context_parallel_attention(q, k, v, group=None, causal: bool = True, scale=N
     k_chunks = gather_chunks(k, group)
     v_chunks = gather_chunks(v, group)
     return context_parallel_local(q, k_chunks, v_chunks, rank, causal=causal, scale=scale)
+
+
+class PeerKV:
+    """K/V chunk buffers that every rank of a group can read in place.
+
+    Each rank writes its own chunk into its buffers; ``views(r)`` returns rank
+    r's buffers as tensors of this process (peer memory over NVLink for
+    r != this rank). The forward kernel's tile loads then read a peer's chunk
+    directly: plain TMA loads, never cluster multicast. Built on torch's
+    symmetric memory; allocate once per (group, chunk shape) and reuse.
+    """
+
+    def __init__(self, shape, dtype=torch.bfloat16, device=None, group=None):
+        import torch.distributed as dist
+        import torch.distributed._symmetric_memory as symm
+        self.group = group if group is not None else dist.group.WORLD
+        self.shape, self.dtype = tuple(shape), dtype
+        self.k = symm.empty(*self.shape, dtype=dtype, device=device)
+        self.v = symm.empty(*self.shape, dtype=dtype, device=device)
+        self._hk = symm.rendezvous(self.k, self.group)
+        self._hv = symm.rendezvous(self.v, self.group)
+
+    def write(self, k: torch.Tensor, v: torch.Tensor) -> None:
+        self.k.copy_(k)
+        self.v.copy_(v)
+
+    def views(self, r: int):
+        return (self._hk.get_buffer(r, self.shape, self.dtype),
+                self._hv.get_buffer(r, self.shape, self.dtype))
+
+
+def _stream_done(t: torch.Tensor) -> None:
+    if t.is_cuda:
+        torch.cuda.current_stream(t.device).synchronize()
+
+
+def context_parallel_attention_peer(q, k, v, peers, group=None, causal: bool = True, scale=None,
+                                    attend=None):
+    """Sequence-sharded attention that reads the other ranks' K/V chunks in place.
+
+    ``peers`` is this group's ``PeerKV`` for the chunk shape. Each rank writes
+    its chunk into its own buffers; once every rank has (barrier), the forward
+    kernel reads each visible chunk from its owner's memory; a second barrier
+    holds the buffers until every rank has finished reading them. Same result
+    as ``context_parallel_attention``. ``attend`` replaces the per-rank
+    attention step (``context_parallel_local``'s signature), for tests.
+    """
+    import torch.distributed as dist
+    rank, world = dist.get_rank(group), dist.get_world_size(group)
+    peers.write(k, v)
+    _stream_done(peers.k)
+    dist.barrier(group=group)                   # every chunk written
+    views = [peers.views(r) for r in range(world)]
+    attend = attend or context_parallel_local
+    out = attend(q, [kv[0] for kv in views], [kv[1] for kv in views], rank, causal=causal,
+                 scale=scale)
+    _stream_done(q)
+    dist.barrier(group=group)                   # every chunk read: buffers may be rewritten
+    return out

@@ -59,3 +59,70 @@ def test_gather_chunks_two_gloo_ranks():
     for rank, vals, shapes in res:
         assert vals == [1.0, 2.0]                    # rank order on every rank
         assert shapes == [(2, 3, 1, 4)] * 2
+
+
+class _SharedPeers:
+    """Stand-in for PeerKV on CPU: every rank's buffers are shared-memory
+    tensors that all ranks can read, as peer memory would be."""
+
+    def __init__(self, bufs_k, bufs_v, rank):
+        self.bufs_k, self.bufs_v = bufs_k, bufs_v
+        self.k, self.v = bufs_k[rank], bufs_v[rank]
+
+    def write(self, k, v):
+        self.k.copy_(k)
+        self.v.copy_(v)
+
+    def views(self, r):
+        return self.bufs_k[r], self.bufs_v[r]
+
+
+def _peer_worker(rank, world, port, bufs_k, bufs_v, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port),
+                      RANK=str(rank), WORLD_SIZE=str(world))
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        from exact_softmax_attention_03_b200.context_parallel import (
+            context_parallel_attention_peer)
+        peers = _SharedPeers(bufs_k, bufs_v, rank)
+
+        def attend(q, k_chunks, v_chunks, r, causal, scale):
+            # what the attention step would read: the first element of every
+            # chunk of its plan
+            return [(s, float(k_chunks[s][0, 0, 0, 0]), float(v_chunks[s][0, 0, 0, 0]))
+                    for s, _ in chunk_plan(r, len(k_chunks), causal)]
+
+        seen = []
+        shape = tuple(bufs_k[rank].shape)
+        for it in range(3):                     # the buffers are reused round after round
+            val = float(10 * it + rank + 1)
+            seen.append(context_parallel_attention_peer(
+                torch.zeros(shape), torch.full(shape, val), torch.full(shape, -val), peers,
+                causal=True, attend=attend))
+        out.put((rank, seen))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_peer_chunks_are_read_in_place_after_every_write(world):
+    ctx = mp.get_context("spawn")
+    shape = (1, 4, 2, 8)
+    bufs_k = [torch.zeros(shape).share_memory_() for _ in range(world)]
+    bufs_v = [torch.zeros(shape).share_memory_() for _ in range(world)]
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_peer_worker, args=(r, world, port, bufs_k, bufs_v, q))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, rounds in res.items():
+        for it, got in enumerate(rounds):
+            want = [(s, float(10 * it + s + 1), -float(10 * it + s + 1)) for s in range(rank + 1)]
+            assert got == want, (rank, it, got)
