@@ -19,7 +19,7 @@ from .attention import (  # noqa: F401
     oracle_decode_paged,
     oracle_probabilities,
     paged_to_contiguous,
-    tiled_attention,
+    key_chunk_attention,
     online_softmax,
     merge_partials,
     brute_force_attention,

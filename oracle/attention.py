@@ -9,8 +9,7 @@ Sources (page title, then section):
 * "Attention Is O(n²): FlashAttention vs Linear Attention", section
   "Why Attention Is O(n²)": the plain operation ``softmax(Q Kᵀ / sqrt(d)) V``;
   section "Wall-Clock Impact of Tiling": the naive reference that materialises
-  the full score matrix, and the tiled online-softmax loop (section
-  "FlashAttention — Same FLOPs, Linear Memory") that reaches the same result.
+  the full score matrix.
 * "Modern Attention: MQA, GQA, FlashAttention, Sliding Window and RoPE",
   section 3 "FlashAttention: exact, but IO-aware" (running max / running
   denominator, worked example on scores [1, 3]) and section 4
@@ -315,15 +314,19 @@ def online_softmax(xs):
     return [math.exp(x - m) / den for x in xs], m, den
 
 
-def tiled_attention(q, k, v, causal=False, window_left=-1, scale=None,
-                    block_q: int = 32, block_k: int = 32):
-    """The tiled loop with running max / running sum / rescaled accumulator.
+def key_chunk_attention(q, k, v, causal=False, window_left=-1, scale=None, chunk: int = 32):
+    """Attention assembled from key chunks, each normalised on its own.
 
-    "Attention Is O(n²) ...", section "FlashAttention — Same FLOPs, Linear
-    Memory": outer loop over query blocks, inner loop over key/value blocks;
-    the accumulator and running sum are rescaled by exp(old_max - new_max) and
-    the output is divided by the running sum at the end. Masked scores are
-    -inf (they contribute exp(-inf) = 0). fp64 throughout.
+    "Chapter 3 ...", section 3.5: a partial softmax state over one set of keys
+    can be merged with the state of another set by rescaling both to their
+    common maximum. Here every chunk of ``chunk`` consecutive keys is treated
+    as its own small attention problem for all query rows at once, giving a
+    normalised output ``O_c`` and its log-sum-exp ``LSE_c`` (a row that sees no
+    key of the chunk has ``O_c = 0``, ``LSE_c = -inf``). The chunks are folded
+    left to right in that normalised form: the merged log-sum-exp is
+    ``log(e^LSE + e^LSE_c)`` and each side's output is weighted by
+    ``e^(its LSE - merged LSE)``, which is the section 3.5 rule with the
+    denominators carried as logarithms. fp64 throughout; no query blocking.
     Returns ``(O [B,Nq,Hq,d], LSE [B,Hq,Nq])``.
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
@@ -332,36 +335,35 @@ def tiled_attention(q, k, v, causal=False, window_left=-1, scale=None,
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     group = Hq // Hkv
-    mask = allowed_mask(Nq, Nk, causal, window_left)
+    keep = allowed_mask(Nq, Nk, causal, window_left)
     O = np.zeros((B, Nq, Hq, d))
     LSE = np.full((B, Hq, Nq), NEG_INF)
     for b in range(B):
         for hq in range(Hq):
-            hk = hq // group
-            for i0 in range(0, Nq, block_q):
-                i1 = min(i0 + block_q, Nq)
-                Qi = q[b, i0:i1, hq]
-                acc = np.zeros((i1 - i0, d))
-                run_max = np.full(i1 - i0, -np.inf)
-                run_sum = np.zeros(i1 - i0)
-                for j0 in range(0, Nk, block_k):
-                    j1 = min(j0 + block_k, Nk)
-                    Sij = scale * (Qi @ k[b, j0:j1, hk].T)
-                    Sij = np.where(mask[i0:i1, j0:j1], Sij, -np.inf)
-                    new_max = np.maximum(run_max, Sij.max(axis=1))
-                    safe = np.where(np.isfinite(new_max), new_max, 0.0)
-                    Pij = np.exp(Sij - safe[:, None])
-                    corr = np.exp(run_max - safe)
-                    acc = acc * corr[:, None] + Pij @ v[b, j0:j1, hk]
-                    run_sum = run_sum * corr + Pij.sum(axis=1)
-                    run_max = new_max
-                ok = run_sum > 0
-                out = np.zeros_like(acc)
-                out[ok] = acc[ok] / run_sum[ok, None]
-                O[b, i0:i1, hq] = out
-                lse = np.full(i1 - i0, -np.inf)
-                lse[ok] = run_max[ok] + np.log(run_sum[ok])
-                LSE[b, hq, i0:i1] = lse
+            kv_head = hq // group
+            out = np.zeros((Nq, d))
+            lse_run = np.full(Nq, NEG_INF)
+            for c0 in range(0, Nk, chunk):
+                cols = slice(c0, min(c0 + chunk, Nk))
+                logits = np.where(keep[:, cols], scale * (q[b, :, hq] @ k[b, cols, kv_head].T),
+                                  NEG_INF)
+                seen = keep[:, cols].any(axis=1)
+                # the chunk's own log-sum-exp and normalised output
+                top = np.where(seen, logits.max(axis=1, initial=NEG_INF), 0.0)
+                mass = np.exp(logits - top[:, None]).sum(axis=1)        # >= 1 where seen
+                lse_c = np.where(seen, top + np.log(np.where(seen, mass, 1.0)), NEG_INF)
+                w_c = np.exp(logits - np.where(seen, lse_c, 0.0)[:, None])   # rows sum to 1
+                out_c = w_c @ v[b, cols, kv_head]
+                # fold: merged log-sum-exp, then both sides reweighted to it
+                both = np.logaddexp(lse_run, lse_c)
+                live = np.isfinite(both)
+                ref = np.where(live, both, 0.0)
+                wa = np.where(np.isfinite(lse_run), np.exp(lse_run - ref), 0.0)
+                wb = np.where(np.isfinite(lse_c), np.exp(lse_c - ref), 0.0)
+                out = np.where(live[:, None], wa[:, None] * out + wb[:, None] * out_c, 0.0)
+                lse_run = both
+            O[b, :, hq] = out
+            LSE[b, hq] = lse_run
     return O, LSE
 
 

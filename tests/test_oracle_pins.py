@@ -4,7 +4,7 @@ Each check compares the oracle with something other than itself: values the
 pages print (fixtures under tests/golden/), exact closed forms for scores that
 are logs of integers, invariants (rows of P sum to 1, constant V, GQA equals
 MHA on repeated K/V, decode equals the last prefill row, window >= N equals
-causal), an independent pure-Python loop, the pages' tiled online-softmax loop,
+causal), an independent pure-Python loop, a key-chunk merge of separately normalised chunks,
 and library routines (torch's float64 SDPA, scipy's logsumexp).
 
 The last test plants plausible mistakes in copies of the oracle (a transposed
@@ -227,15 +227,14 @@ def test_decode_equals_last_row_of_causal_prefill():
             assert np.allclose(Ld[b], Lp[0, :, s - 1], atol=1e-13)
 
 
-def test_tiled_loop_equals_materialising_oracle():
+def test_key_chunk_merge_equals_materialising_oracle():
     rng = np.random.default_rng(6)
     q = rng.standard_normal((2, 70, 4, 16)) * 3.0
     k = rng.standard_normal((2, 90, 2, 16)) * 3.0
     v = rng.standard_normal((2, 90, 2, 16))
     for causal, wl in [(False, -1), (True, -1), (True, 17), (False, 40)]:
         O1, L1 = oracle.oracle_attention(q, k, v, causal=causal, window_left=wl)
-        O2, L2 = oracle.tiled_attention(q, k, v, causal=causal, window_left=wl,
-                                        block_q=32, block_k=32)
+        O2, L2 = oracle.key_chunk_attention(q, k, v, causal=causal, window_left=wl, chunk=32)
         assert np.allclose(O1, O2, atol=1e-12, rtol=0)
         assert np.allclose(L1, L2, atol=1e-12, rtol=0)
 

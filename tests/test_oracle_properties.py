@@ -6,7 +6,7 @@ included), windows down to 0 and random inputs. The NumPy oracle must agree
 with the independent formulations the oracle module carries:
 
 - the pure-Python loops;
-- the pages' tiled online-softmax loop, with random block sizes;
+- the key-chunk merge (section 3.5 rule), with random chunk sizes;
 - decode as the last causal row;
 - the merge rule over a random split of the keys;
 - the backward identities (a head's key gradients sum to zero; its value
@@ -64,11 +64,11 @@ def test_numpy_oracle_equals_pure_python_loops(p):
 
 
 @SETTINGS
-@given(problems(), st.integers(1, 5), st.integers(1, 5))
-def test_tiled_loop_equals_materialised(p, bq, bk):
+@given(problems(), st.integers(1, 5))
+def test_key_chunk_merge_equals_materialised(p, ck):
     q, k, v, causal, wl = p
     O, L = oracle.oracle_attention(q, k, v, causal=causal, window_left=wl)
-    Ot, Lt = oa.tiled_attention(q, k, v, causal=causal, window_left=wl, block_q=bq, block_k=bk)
+    Ot, Lt = oa.key_chunk_attention(q, k, v, causal=causal, window_left=wl, chunk=ck)
     _same(O, Ot)
     _same(L, Lt)
 
