@@ -46,6 +46,18 @@ def _need(t: torch.Tensor, name: str, dtype, ndim: int):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _shape(t: torch.Tensor, name: str, shape):
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _same_device(ref: torch.Tensor, *named):
+    """Every operand on the device of ``ref`` (the kernels read them all there)."""
+    for t, name in named:
+        if t is not None and t.device != ref.device:
+            raise ValueError(f"{name} is on {t.device}, expected {ref.device}")
+
+
 def _fwd(q, k, v, o, lse, causal, window_left, scale, stream, f32o):
     _need(q, "q", torch.bfloat16, 4)
     _need(k, "k", torch.bfloat16, 4)
@@ -64,6 +76,7 @@ def _fwd(q, k, v, o, lse, causal, window_left, scale, stream, f32o):
         _need(lse, "lse", torch.float32, 3)
         if tuple(lse.shape) != (B, Hq, Nq):
             raise ValueError("lse must be [B, Hq, Nq]")
+    _same_device(q, (k, "k"), (v, "v"), (o, "o"), (lse, "lse"))
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     fn = load().attn_fwd_f32o if f32o else load().attn_fwd
@@ -108,8 +121,12 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqle
     if o is None:
         o = torch.empty((total_q, Hq, d), dtype=torch.bfloat16, device=q.device)
     _need(o, "o", torch.bfloat16, 3)
+    _shape(o, "o", (total_q, Hq, d))
     if lse is not None:
         _need(lse, "lse", torch.float32, 2)
+        _shape(lse, "lse", (Hq, total_q))
+    _same_device(q, (k, "k"), (v, "v"), (cu_seqlens_q, "cu_seqlens_q"),
+                 (cu_seqlens_k, "cu_seqlens_k"), (o, "o"), (lse, "lse"))
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     check(load().attn_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
@@ -140,11 +157,20 @@ def attn_bwd(q, k, v, o, lse, dout, causal=False, window_left=-1, scale=None, dq
     _, Nk, Hkv, _ = k.shape
     if o.shape != q.shape or dout.shape != q.shape or v.shape != k.shape:
         raise ValueError("o and dout must be shaped like q, v like k")
+    if k.shape[0] != B or k.shape[3] != d:
+        raise ValueError("k, v must be [B, Nk, Hkv, d] matching q")
+    _shape(lse, "lse", (B, Hq, Nq))
+    for t, n, like in ((dq, "dq", q), (dk, "dk", k), (dv, "dv", v)):
+        if t is not None:
+            _need(t, n, torch.bfloat16, 4)
+            _shape(t, n, like.shape)
+    if workspace is not None and not isinstance(workspace, torch.Tensor):
+        raise TypeError("workspace must be a torch.Tensor")
+    _same_device(q, (k, "k"), (v, "v"), (o, "o"), (lse, "lse"), (dout, "dout"), (dq, "dq"),
+                 (dk, "dk"), (dv, "dv"), (workspace, "workspace"))
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
-        _need(t, n, torch.bfloat16, 4)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     need = attn_bwd_workspace_bytes(B, Hq, Nq, d)
@@ -169,8 +195,11 @@ def attn_merge(o_parts, lse_parts, o=None, lse=None, stream=None):
     if o is None:
         o = torch.empty((B, Nq, Hq, d), dtype=torch.bfloat16, device=o_parts.device)
     _need(o, "o", torch.bfloat16, 4)
+    _shape(o, "o", (B, Nq, Hq, d))
     if lse is not None:
         _need(lse, "lse", torch.float32, 3)
+        _shape(lse, "lse", (B, Hq, Nq))
+    _same_device(o_parts, (lse_parts, "lse_parts"), (o, "o"), (lse, "lse"))
     check(load().attn_merge(o_parts.data_ptr(), lse_parts.data_ptr(), R, o.data_ptr(),
                             lse.data_ptr() if lse is not None else None, B, Nq, Hq, d,
                             _stream_handle(stream)))
@@ -199,16 +228,21 @@ def attn_decode(q, k_cache, v_cache, o=None, lse=None, seqlens=None, window_left
     if o is None:
         o = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q.device)
     _need(o, "o", torch.bfloat16, 3)
+    _shape(o, "o", (B, Hq, d))
     if lse is not None:
         _need(lse, "lse", torch.float32, 2)
+        _shape(lse, "lse", (B, Hq))
     if seqlens is not None:
         _need(seqlens, "seqlens", torch.int32, 1)
+        _shape(seqlens, "seqlens", (B,))
+    _same_device(q, (k_cache, "k_cache"), (v_cache, "v_cache"), (o, "o"), (lse, "lse"),
+                 (seqlens, "seqlens"), (workspace, "workspace"))
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     need = attn_decode_workspace_bytes(B, Hq, d, num_splits, Lmax)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
-    if not workspace.is_cuda:
+    if not isinstance(workspace, torch.Tensor) or not workspace.is_cuda:
         raise ValueError("workspace must be a CUDA tensor")
     ws_bytes = workspace.numel() * workspace.element_size()
     check(load().attn_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), o.data_ptr(),
@@ -243,16 +277,21 @@ def attn_decode_paged(q, k_pages, v_pages, block_table, o=None, lse=None, seqlen
     if o is None:
         o = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q.device)
     _need(o, "o", torch.bfloat16, 3)
+    _shape(o, "o", (B, Hq, d))
     if lse is not None:
         _need(lse, "lse", torch.float32, 2)
+        _shape(lse, "lse", (B, Hq))
     if seqlens is not None:
         _need(seqlens, "seqlens", torch.int32, 1)
+        _shape(seqlens, "seqlens", (B,))
+    _same_device(q, (k_pages, "k_pages"), (v_pages, "v_pages"), (block_table, "block_table"),
+                 (o, "o"), (lse, "lse"), (seqlens, "seqlens"), (workspace, "workspace"))
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     need = attn_decode_workspace_bytes(B, Hq, d, num_splits, pages_per_seq * page_size)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
-    if not workspace.is_cuda:
+    if not isinstance(workspace, torch.Tensor) or not workspace.is_cuda:
         raise ValueError("workspace must be a CUDA tensor")
     ws_bytes = workspace.numel() * workspace.element_size()
     check(load().attn_decode_paged(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(), o.data_ptr(),
@@ -288,10 +327,15 @@ def attn_decode_noalloc(q, k_cache, v_cache, o=None, lse=None, seqlens=None, win
     if o is None:
         o = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q.device)
     _need(o, "o", torch.bfloat16, 3)
+    _shape(o, "o", (B, Hq, d))
     if lse is not None:
         _need(lse, "lse", torch.float32, 2)
+        _shape(lse, "lse", (B, Hq))
     if seqlens is not None:
         _need(seqlens, "seqlens", torch.int32, 1)
+        _shape(seqlens, "seqlens", (B,))
+    _same_device(q, (k_cache, "k_cache"), (v_cache, "v_cache"), (o, "o"), (lse, "lse"),
+                 (seqlens, "seqlens"))
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     check(load().attn_decode_noalloc(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),

@@ -95,6 +95,15 @@ class PeerKV:
         self._hv = symm.rendezvous(self.v, self.group)
 
     def write(self, k: torch.Tensor, v: torch.Tensor) -> None:
+        """Copy this rank's chunk in. The chunk must match the buffers exactly:
+        a copy that broadcast a smaller chunk would give every rank wrong data."""
+        for t, name in ((k, "k"), (v, "v")):
+            if tuple(t.shape) != self.shape:
+                raise ValueError(f"{name} chunk has shape {tuple(t.shape)}, buffers hold {self.shape}")
+            if t.dtype != self.dtype:
+                raise ValueError(f"{name} chunk is {t.dtype}, buffers hold {self.dtype}")
+            if t.device != self.k.device:
+                raise ValueError(f"{name} chunk is on {t.device}, buffers are on {self.k.device}")
         self.k.copy_(k)
         self.v.copy_(v)
 
@@ -118,16 +127,21 @@ def context_parallel_attention_peer(q, k, v, peers, group=None, causal: bool = T
     holds the buffers until every rank has finished reading them. Same result
     as ``context_parallel_attention``. ``attend`` replaces the per-rank
     attention step (``context_parallel_local``'s signature), for tests.
+    If the attention step raises on one rank, that rank still takes the second
+    barrier before the error propagates, so the other ranks are not left
+    waiting for it.
     """
     import torch.distributed as dist
     rank, world = dist.get_rank(group), dist.get_world_size(group)
     peers.write(k, v)
     _stream_done(peers.k)
     dist.barrier(group=group)                   # every chunk written
-    views = [peers.views(r) for r in range(world)]
     attend = attend or context_parallel_local
-    out = attend(q, [kv[0] for kv in views], [kv[1] for kv in views], rank, causal=causal,
-                 scale=scale)
-    _stream_done(q)
-    dist.barrier(group=group)                   # every chunk read: buffers may be rewritten
+    try:
+        views = [peers.views(r) for r in range(world)]
+        out = attend(q, [kv[0] for kv in views], [kv[1] for kv in views], rank, causal=causal,
+                     scale=scale)
+        _stream_done(q)
+    finally:
+        dist.barrier(group=group)               # every chunk read: buffers may be rewritten
     return out

@@ -9,8 +9,10 @@ partial results in the library's own fixed device scratch instead.
 These tests call the entry point through the C ABI (ctypes, raw pointers) and
 check its results against the ordinary attn_decode with a caller workspace,
 within the tolerances of the other parity tests, on two calls in a row (the
-second call finds the first call's leftovers in the shared scratch). The file
-is named so that pytest collects it last.
+second call finds the first call's leftovers in the shared scratch). Both
+calls are also compared with the fp64 oracle directly: the ragged case whole,
+the full decode workload on a sample of its sequences. The file is named so
+that pytest collects it last.
 """
 
 import ctypes
@@ -107,3 +109,13 @@ def test_noalloc_matches_workspace_decode_on_two_calls_in_a_row(lib):
     torch.cuda.synchronize()
     _close(o1, r1, l1, rl1)
     _close(o2, r2, l2, rl2)
+    # and against the oracle itself, not only through the other CUDA path
+    import oracle
+    from parity import assert_close
+    sel = [0, 21, 42, 63]                            # sequences of the decode workload
+    O1, L1 = oracle.oracle_decode(first["q"][sel].cpu(), first["k"][sel].cpu(),
+                                  first["v"][sel].cpu())
+    assert_close(o1[sel], O1, l1[sel], L1, what="noalloc decode workload (sampled sequences)")
+    O2, L2 = oracle.oracle_decode(second["q"].cpu(), second["k"].cpu(), second["v"].cpu(),
+                                  seqlens=second["sl"].cpu(), window_left=300)
+    assert_close(o2, O2, l2, L2, what="noalloc ragged, window 300, 5 splits")
