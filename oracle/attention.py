@@ -53,7 +53,7 @@ def _f64(x) -> np.ndarray:
     return np.asarray(x, dtype=np.float64)
 
 
-def allowed_mask(Nq: int, Nk: int, causal: bool, window_left: int) -> np.ndarray:
+def allowed_mask(Nq: int, Nk: int, causal: bool, window_left: int, rows=None) -> np.ndarray:
     """Boolean ``[Nq, Nk]`` mask of the (query, key) pairs that take part.
 
     Query row ``i`` sits at key position ``qpos = i + Nk - Nq`` (bottom-right
@@ -61,11 +61,13 @@ def allowed_mask(Nq: int, Nk: int, causal: bool, window_left: int) -> np.ndarray
     ``j >= qpos - window_left`` (if ``window_left >= 0``). With ``Nq = Nk = 8``,
     ``causal`` and ``window_left = 2`` this is the "last W = 3 tokens" diagram
     of "Modern Attention ...", section 4 "Sliding-window attention".
+    ``rows`` (optional) selects query rows: the result is then
+    ``[len(rows), Nk]``, the same rows of the full mask.
     """
-    i = np.arange(Nq)[:, None]
+    i = (np.arange(Nq) if rows is None else np.asarray(rows, dtype=np.int64))[:, None]
     j = np.arange(Nk)[None, :]
     qpos = i + (Nk - Nq)
-    ok = np.ones((Nq, Nk), dtype=bool)
+    ok = np.ones((i.shape[0], Nk), dtype=bool)
     if causal:
         ok &= j <= qpos
     if window_left is not None and window_left >= 0:
@@ -141,7 +143,7 @@ def oracle_attention_rows(q, k, v, b: int, hq: int, rows, causal: bool = False,
         scale = 1.0 / math.sqrt(d)
     rows = np.asarray(rows, dtype=np.int64)
     hk = hq // (Hq // Hkv)
-    mask = allowed_mask(Nq, Nk, causal, window_left)[rows]
+    mask = allowed_mask(Nq, Nk, causal, window_left, rows=rows)
     o, lse, _ = _head_attention(q[b, rows, hq], k[b, :, hk], v[b, :, hk], scale, mask)
     return o, lse
 

@@ -46,14 +46,16 @@ def test_sharded_sequence_equals_whole(R, C, Hq, Hkv, d, causal):
     assert_close(torch.cat(outs, dim=1), O, torch.cat(lses, dim=2), L, what=(R, C, causal))
 
 
-@pytest.mark.parametrize("R,d", [(3, 128), (5, 64), (20, 128)])
-def test_merge_kernel_against_merge_rule(R, d):
+@pytest.mark.parametrize("R,d,Nq", [(3, 128, 17), (5, 64, 17), (20, 128, 17), (1, 128, 70),
+                                    (2, 64, 70), (4, 128, 70), (8, 128, 33), (9, 64, 64),
+                                    (64, 128, 40)])
+def test_merge_kernel_against_merge_rule(R, d, Nq):
     import exact_softmax_attention_03_b200 as ea
     g = torch.Generator().manual_seed(7)
-    B, Nq, H = 2, 17, 4
+    B, H = 2, 4
     op = torch.randn(R, B, Nq, H, d, generator=g)
     lp = torch.randn(R, B, H, Nq, generator=g) * 3
-    lp[1, 0, 2, 5] = -float("inf")                 # one part saw no key for this row
+    lp[min(1, R - 1), 0, 2, 5] = -float("inf")     # one part saw no key for this row
     lp[:, 1, 3, 7] = -float("inf")                 # no part saw a key
     o, lse = ea.attn_merge(op.cuda(), lp.cuda(), lse=torch.empty(B, H, Nq, device="cuda"))
     assert ea.attn_device_status() == 0

@@ -121,17 +121,49 @@ def test_constant_v_gives_constant_output():
 FULL = [ai.MHA_2K, ai.MHA_8K, ai.GQA_SWA_32K]
 
 
+def _head(t, b, h):
+    return t[b:b + 1, :, h:h + 1]
+
+
 @pytest.mark.parametrize("w", FULL, ids=lambda w: w.name)
-def test_full_size_sampled_rows(w):
+def test_full_size_whole_head_and_late_rows(w):
+    """One launch at the full workload size, in the bench's configuration.
+
+    * One whole (batch, head) is compared element by element with the oracle
+      (every row block of that head, so every position in the work order);
+      at N = 32768, where one head costs the fp64 oracle about a minute, two
+      spans of 512 rows of it (the middle and the end).
+    * The shortest causal row blocks run last in the kernel's work order
+      (longest rows first); rows of the first 256 and of the last 256 query
+      positions are sampled on 12 more heads, plus 24 rows anywhere.
+    """
     q, k, v = ai.make_for(w)
     o, lse = run_fwd(q, k, v, w.causal, w.window_left)
     assert torch.isfinite(o.float()).all()
     assert torch.isfinite(lse).all()
+    G = w.Hq // w.Hkv
+    b, hq = w.B - 1, w.Hq - 1
+    if w.Nq * w.Nk <= 8192 * 8192:
+        O, L = oracle.oracle_attention(_head(q, b, hq), _head(k, b, hq // G),
+                                       _head(v, b, hq // G), causal=w.causal,
+                                       window_left=w.window_left)
+        assert_close(o[b:b + 1, :, hq:hq + 1], O, lse[b:b + 1, hq:hq + 1], L,
+                     what=(w.name, "whole head", b, hq))
+    else:
+        rows = list(range(w.Nq // 2, w.Nq // 2 + 512)) + list(range(w.Nq - 512, w.Nq))
+        O, L = oracle.oracle_attention_rows(_head(q, b, hq), _head(k, b, hq // G),
+                                            _head(v, b, hq // G), 0, 0, rows, causal=w.causal,
+                                            window_left=w.window_left)
+        assert_close(o[b, rows, hq], O, lse[b, hq, rows], L, what=(w.name, "row spans", b, hq))
     g = torch.Generator().manual_seed(99)
-    for b, hq in [(0, 0), (w.B - 1, w.Hq - 1), (int(torch.randint(w.B, (1,), generator=g)),
-                                                int(torch.randint(w.Hq, (1,), generator=g)))]:
-        rows = sample_rows(w.Nq, 24, seed=b * 1000 + hq)
-        O, L = oracle.oracle_attention_rows(q, k, v, b, hq, rows, causal=w.causal,
+    for i in range(12):
+        b = int(torch.randint(w.B, (1,), generator=g))
+        hq = int(torch.randint(w.Hq, (1,), generator=g))
+        early = torch.randint(0, 256, (8,), generator=g).tolist()
+        late = torch.randint(w.Nq - 256, w.Nq, (4,), generator=g).tolist()
+        rows = sorted(set(early + late + sample_rows(w.Nq, 24, seed=1000 * b + hq)))
+        O, L = oracle.oracle_attention_rows(_head(q, b, hq), _head(k, b, hq // G),
+                                            _head(v, b, hq // G), 0, 0, rows, causal=w.causal,
                                             window_left=w.window_left)
         assert_close(o[b, rows, hq], O, lse[b, hq, rows], L, what=(w.name, b, hq))
 

@@ -405,3 +405,12 @@ def test_unmutated_control_passes_all_pins(golden):
     assert pin_page_worked_example(attn, golden)
     assert pin_gqa_is_repeated_mha(attn, np.random.default_rng(4))
     assert pin_window_pattern(mask_fn, golden)
+
+
+def test_mask_of_selected_rows_is_those_rows_of_the_full_mask():
+    rng = np.random.default_rng(11)
+    for Nq, Nk, causal, wl in [(37, 37, True, -1), (20, 50, True, 7), (50, 20, True, -1),
+                               (30, 30, False, 4), (9, 9, False, -1)]:
+        full = oracle.allowed_mask(Nq, Nk, causal, wl)
+        rows = sorted(rng.choice(Nq, size=min(Nq, 11), replace=False).tolist())
+        assert (oracle.allowed_mask(Nq, Nk, causal, wl, rows=rows) == full[rows]).all()
