@@ -2,12 +2,18 @@
 """Benchmark of the exact-attention hot path on B200 (one JSON line on rank 0).
 
 A step is one pass of the hot path over one batch of synthetic input:
-  * prefill: one attn_fwd call on the MHA causal prefill workload
-    (B=4, Hq=Hkv=32, N=2048, d=128, bf16 in/out, fp32 LSE) — the headline
-    `value`, in mask-adjusted TFLOP/s;
+  * prefill: one attn_fwd call on the headline workload, by default the MHA
+    causal prefill at the page-1 shape (B=4, Hq=Hkv=32, N=8192, d=128, bf16
+    in/out, fp32 LSE) — the headline `value`, in mask-adjusted TFLOP/s;
+  * the two other prefill workloads as their own legs ("prefill_legs"): MHA
+    causal N=2048 and GQA sliding window N=32768 (Hq=32, Hkv=8,
+    window_left=4096), each with its own roofline;
   * decode: one attn_decode call (split + combine kernels) on the GQA decode
     workload (B=64, L=8192, Hq=32, Hkv=8, d=128), reported under "decode" in
-    KV-read GB/s, timed over the same number of steps.
+    KV-read GB/s;
+  * the later rows (backward, merge, packed prefill, paged decode) as legs.
+Each leg is timed over the same number of steps; mean, median and min are
+reported (the headline value uses the mean: total time over K steps).
 
 Timing: W untimed warm-up steps, then K steps; each kernel is bracketed by
 CUDA events on the launching stream, preceded by an L2 flush (256 MiB
@@ -17,7 +23,8 @@ With N > 1 every rank runs its own independent batch (no collective in the
 data path): weak scaling.
 
 `--impl reference` times the fp64 CPU oracle instead (the only other
-implementation of this path), one bounded per-head sample per step.
+implementation of this path): each step is one block of 512 query rows of one
+(batch, head) of the headline workload.
 """
 
 from __future__ import annotations
@@ -52,6 +59,8 @@ KERNEL_SOURCES = {
                      for f in ("sm100_ptx.cuh", "decode_kernels.cuh")],
     "bwd_main_kernel": ["exact_softmax_attention_03_b200/csrc/" + f
                         for f in ("sm100_ptx.cuh", "backward_kernels.cuh")],
+    "merge": ["exact_softmax_attention_03_b200/csrc/" + f
+              for f in ("sm100_ptx.cuh", "merge_kernel.cuh")],
 }
 
 
@@ -61,8 +70,10 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["mha2k", "mha8k", "gqa32k"], default="mha2k",
-                    help="prefill workload (default: the MHA causal prefill at N=2048)")
+    ap.add_argument("--workload", choices=["mha2k", "mha8k", "gqa32k"], default="mha8k",
+                    help="headline prefill workload (default: MHA causal N=8192, the page-1 shape)")
+    ap.add_argument("--only-headline", action="store_true",
+                    help="skip the other prefill workloads' legs")
     ap.add_argument("--decode-splits", type=int, default=0)
     ap.add_argument("--batch", type=int, default=0,
                     help="override the prefill batch (profiling a smaller case only)")
@@ -213,7 +224,7 @@ def whole_job_rate(units_per_rank: float, ms_max: float, world: int) -> float:
 
 # ------------------------------------------------------------------ timing --
 
-def timed_kernel_loop(fn, steps, warmup, world, flush=None, sampler=None):
+def timed_kernel_loop(fn, steps, warmup, world, flush=None):
     """Per-step CUDA-event times (ms) of fn() on the current stream; returns
     (times, launches of this library inside the timed region)."""
     import exact_softmax_attention_03_b200 as ea
@@ -222,29 +233,31 @@ def timed_kernel_loop(fn, steps, warmup, world, flush=None, sampler=None):
             flush()
         fn()
     torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(steps)]
     barrier(world)
     torch.cuda.synchronize()
-    if sampler is not None:
-        sampler.start()
     n0 = ea.attn_launch_count()
     for s, e in ev:
         if flush is not None:
             flush()
         torch.cuda._sleep(100_000)              # hold the stream while the launch is queued
-        s.record()
+        s.record(stream)
         fn()
-        e.record()
+        e.record(stream)
     torch.cuda.synchronize()
     n1 = ea.attn_launch_count()
     barrier(world)
-    if sampler is not None:
-        sampler.stop()
     status = ea.attn_device_status()
     if status != 0:
         raise RuntimeError(f"device status {status}: {ea.attn_last_error()}")
     return [s.elapsed_time(e) for s, e in ev], n1 - n0
+
+
+def time_stats(times):
+    """mean / median / min of per-step times (ms)."""
+    return {"mean": statistics.mean(times), "median": statistics.median(times), "min": min(times)}
 
 
 def e2e_loop(step_fn, steps, warmup):
@@ -265,44 +278,70 @@ def e2e_loop(step_fn, steps, warmup):
 
 # ------------------------------------------------------------ cpu baseline --
 
-def blas_threads():
+def blas_info():
+    """(threads, vendor string) of the BLAS NumPy calls into."""
     try:
         from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
-        return max(n) if n else 1
+        infos = [i for i in threadpool_info() if i.get("user_api") == "blas"]
+        if infos:
+            i = max(infos, key=lambda x: x.get("num_threads", 0))
+            vendor = f"{i.get('internal_api', '?')} {i.get('version', '')}".strip()
+            return int(i.get("num_threads", 1)), vendor
     except Exception:
-        return os.cpu_count() or 1
+        pass
+    return os.cpu_count() or 1, "unknown"
 
 
-def oracle_prefill_sample(w, budget_s, q, k, v):
-    """Time the oracle on whole (b, head) problems until ~budget_s of CPU work."""
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+ROW_BLOCK = 512
+
+
+def oracle_row_blocks(w):
+    """The sample unit of the CPU legs: (b, head, first row) of 512-row blocks,
+    spread over the rows so that short and long causal rows both appear."""
+    blocks = list(range(0, w.Nq, ROW_BLOCK))
+    order = blocks[::-2] + blocks[-2::-2]                   # longest and shortest rows mixed
+    return [(b, h, r0) for b in range(w.B) for h in range(w.Hq) for r0 in order]
+
+
+def oracle_block(w, q, k, v, b, hq, r0):
+    """One oracle call on rows [r0, r0 + 512) of one (batch, head); its FLOPs.
+
+    The oracle is handed that head's slices only (it upcasts what it is given)."""
     import oracle
-    G = w.Hq // w.Hkv
-    pairs_per_head = metrics.allowed_pairs(w.Nq, w.Nk, w.causal, w.window_left)
-    flops = 0.0
-    heads = 0
+    rows = list(range(r0, min(r0 + ROW_BLOCK, w.Nq)))
+    hk = hq // (w.Hq // w.Hkv)
+    oracle.oracle_attention_rows(q[b:b + 1, :, hq:hq + 1], k[b:b + 1, :, hk:hk + 1],
+                                 v[b:b + 1, :, hk:hk + 1], 0, 0, rows, causal=w.causal,
+                                 window_left=w.window_left)
+    per_row = metrics.allowed_pairs_per_row(w.Nq, w.Nk, w.causal, w.window_left)
+    return 4.0 * w.d * float(per_row[rows[0]:rows[-1] + 1].sum())
+
+
+def cpu_baseline_block(w, q, k, v, budget_s):
+    """The fp64 oracle timed on 512-row blocks of the workload for ~budget_s."""
+    units = oracle_row_blocks(w)
+    flops, n = 0.0, 0
     t0 = time.perf_counter()
-    for b in range(w.B):
-        for hq in range(w.Hq):
-            hk = hq // G
-            oracle.oracle_attention(q[b:b + 1, :, hq:hq + 1], k[b:b + 1, :, hk:hk + 1],
-                                    v[b:b + 1, :, hk:hk + 1], causal=w.causal,
-                                    window_left=w.window_left)
-            flops += 4.0 * w.d * pairs_per_head
-            heads += 1
-            if time.perf_counter() - t0 >= budget_s:
-                break
-        if time.perf_counter() - t0 >= budget_s:
-            break
+    while time.perf_counter() - t0 < budget_s and n < len(units):
+        flops += oracle_block(w, q, k, v, *units[n])
+        n += 1
     dt = time.perf_counter() - t0
-    return flops / dt / 1e12, heads, dt
-
-
-def cpu_baseline_block(w, q, k, v, budget_s=12.0):
-    tflops, heads, dt = oracle_prefill_sample(w, budget_s, q, k, v)
-    return {"value": tflops, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"fp64 NumPy oracle on {heads} whole (batch, head) problems of "
-                      f"'{w.name}' ({dt:.1f} s), same mask-adjusted FLOP count"}
+    threads, vendor = blas_info()
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"fp64 NumPy oracle on {n} blocks of {ROW_BLOCK} query rows of "
+                      f"'{w.name}' ({dt:.1f} s of CPU work), same mask-adjusted FLOP count",
+            "host_cpus": os.cpu_count(), "cpu_model": cpu_model(), "blas": vendor}
 
 
 # --------------------------------------------------------------- reference --
@@ -312,35 +351,28 @@ def run_reference(args, world, rank):
         return
     w = PREFILL[args.workload]
     q, k, v = ai.make_for(w)
-    import oracle
-    G = w.Hq // w.Hkv
-    flops_head = 4.0 * w.d * metrics.allowed_pairs(w.Nq, w.Nk, w.causal, w.window_left)
-    heads = [(b, h) for b in range(w.B) for h in range(w.Hq)]
-
-    def step(i):
-        b, hq = heads[i % len(heads)]
-        hk = hq // G
-        oracle.oracle_attention(q[b:b + 1, :, hq:hq + 1], k[b:b + 1, :, hk:hk + 1],
-                                v[b:b + 1, :, hk:hk + 1], causal=w.causal, window_left=w.window_left)
-
+    units = oracle_row_blocks(w)
     for i in range(args.warmup):
-        step(i)
+        oracle_block(w, q, k, v, *units[i % len(units)])
+    flops = 0.0
     t0 = time.perf_counter()
     for i in range(args.steps):
-        step(i)
-    dt = (time.perf_counter() - t0) / args.steps
-    value = flops_head / dt / 1e12
+        flops += oracle_block(w, q, k, v, *units[(args.warmup + i) % len(units)])
+    dt = time.perf_counter() - t0
+    value = flops / dt / 1e12
+    threads, vendor = blas_info()
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "seq_len": w.Nq,
                    "d": w.d, "causal": w.causal, "window_left": w.window_left,
-                   "step": "one whole (batch, head) problem per step"},
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(),
-                         "kind": "oracle",
-                         "sample": "one (batch, head) problem per step, fp64 NumPy oracle"},
+                   "step": f"one block of {ROW_BLOCK} query rows of one (batch, head)"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{args.steps} blocks of {ROW_BLOCK} query rows, fp64 NumPy "
+                                   f"oracle, mask-adjusted FLOPs",
+                         "host_cpus": os.cpu_count(), "cpu_model": cpu_model(), "blas": vendor},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -348,6 +380,56 @@ def run_reference(args, world, rank):
 
 
 # -------------------------------------------------------------------- ours --
+
+def tensor_roofline(achieved, peaks, peak_src, kernel, traffic, alg_bytes=None):
+    peak_t = peaks["bf16_tflops"]
+    r = {"bound": "tensor", "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
+         "frac": achieved / peak_t, "peak_source": f"{peak_src} bf16_tflops (burst)",
+         "kernel": kernel, "traffic": traffic}
+    if alg_bytes is not None:
+        r["algorithmic_bytes"] = alg_bytes
+    return r
+
+
+def hbm_roofline(achieved, peaks, peak_src, kernel, traffic, alg_bytes):
+    return {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "peak_source": f"{peak_src} hbm_gbs",
+            "kernel": kernel, "algorithmic_bytes": alg_bytes, "traffic": traffic}
+
+
+def prefill_leg(ea, key, w, args, world, rank, dev, flush, peaks, peak_src, resized=False):
+    """Time attn_fwd on one prefill workload; returns (leg dict, device tensors)."""
+    q_h, k_h, v_h = ai.make_for(w, seed=shard_seed(rank))
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    o = torch.empty((w.B, w.Nq, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=dev)
+
+    def fwd():
+        ea.attn_fwd(q, k, v, o=o, lse=lse, causal=w.causal, window_left=w.window_left)
+
+    times, launches = timed_kernel_loop(fwd, args.steps, args.warmup, world, flush)
+    st = time_stats(times)
+    ms_max = max_over_ranks(st["mean"], world)
+    flops = metrics.attn_flops(w.B, w.Hq, w.Nq, w.Nk, w.d, w.causal, w.window_left)
+    tiles = metrics.executed_tiles(w.Nq, w.Nk, w.causal, w.window_left) * w.B * w.Hq
+    leg = {
+        "workload": w.name, "key": key,
+        "config": {"B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "seq_len": w.Nq, "d": w.d,
+                   "causal": w.causal, "window_left": w.window_left},
+        "value": whole_job_rate(flops, ms_max, world) / 1e12, "unit": "TFLOP/s",
+        "ms_per_step": ms_max, "ms": st,
+        "flops_per_step": flops,
+        "tflops_at_median": flops / (st["median"] * 1e-3) / 1e12,
+        "tile_tflops": tiles * 4.0 * 128 * 128 * w.d / (st["mean"] * 1e-3) / 1e12,
+        "roofline": tensor_roofline(flops / (st["mean"] * 1e-3) / 1e12, peaks, peak_src,
+                                    "attn_fwd_kernel<128,false>",
+                                    recorded_traffic("attn_fwd_kernel", key, resized),
+                                    metrics.attn_fwd_bytes(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d)),
+        "gpu_launches": launches,
+    }
+    leg["pct_bf16_peak"] = 100.0 * leg["roofline"]["frac"]
+    return leg, (q_h, k_h, v_h, q, k, v, o, lse)
+
 
 def run_ours(args, world, rank, local):
     import exact_softmax_attention_03_b200 as ea
@@ -357,33 +439,40 @@ def run_ours(args, world, rank, local):
     torch.cuda.set_device(dev)
     peaks, peak_src = load_peaks()
     sampler = ClockSampler(torch.cuda.current_device() if world == 1 else local)
-
-    w = PREFILL[args.workload]
-    if args.batch:
-        w = dataclasses.replace(w, B=args.batch, name=f"{w.name} [batch {args.batch}]")
-    q_h, k_h, v_h = ai.make_for(w, seed=shard_seed(rank))
-    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
-    o = torch.empty((w.B, w.Nq, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
-    lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=dev)
     flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
     def flush():
         flush_buf.zero_()
 
-    def fwd():
-        ea.attn_fwd(q, k, v, o=o, lse=lse, causal=w.causal, window_left=w.window_left)
+    resized = bool(args.batch)
+    w = PREFILL[args.workload]
+    if args.batch:
+        w = dataclasses.replace(w, B=args.batch, name=f"{w.name} [batch {args.batch}]")
 
-    times, launches = timed_kernel_loop(fwd, args.steps, args.warmup, world, flush, sampler)
-    ms = statistics.mean(times)
-    ms_max = max_over_ranks(ms, world)
-    flops = metrics.attn_flops(w.B, w.Hq, w.Nq, w.Nk, w.d, w.causal, w.window_left)
-    value = whole_job_rate(flops, ms_max, world) / 1e12
-    achieved = flops / (ms * 1e-3) / 1e12
-    tiles = metrics.executed_tiles(w.Nq, w.Nk, w.causal, w.window_left) * w.B * w.Hq
-    clocks = sampler.summary()
+    sampler.start()
+    # ---- headline prefill
+    head, (q_h, k_h, v_h, q, k, v, o, lse) = prefill_leg(
+        ea, args.workload, w, args, world, rank, dev, flush, peaks, peak_src, resized)
+    launches = head["gpu_launches"]
 
-    # backward leg on the same workload: dQ, dK, dV from the forward's O and LSE
-    # (2.5x the forward's mask-adjusted FLOPs: five products instead of two)
+    # ---- the other prefill workloads, each its own leg
+    legs = []
+    if not args.only_headline:
+        for key in ("mha2k", "mha8k", "gqa32k"):
+            if key == args.workload:
+                continue
+            wl = PREFILL[key]
+            if args.batch and wl.B > 1:
+                wl = dataclasses.replace(wl, B=min(wl.B, args.batch),
+                                         name=f"{wl.name} [batch {min(wl.B, args.batch)}]")
+            leg, tensors = prefill_leg(ea, key, wl, args, world, rank, dev, flush, peaks,
+                                       peak_src, resized)
+            legs.append(leg)
+            del tensors
+
+    # ---- backward on the headline workload: dQ, dK, dV from the forward's O and
+    # LSE (2.5x the forward's mask-adjusted FLOPs: five products instead of two)
+    flops = head["flops_per_step"]
     do_h = ai.make_dout(w.B, w.Nq, w.Hq, w.d, seed=shard_seed(rank) + 21)
     dout = do_h.to(dev)
     ea.attn_fwd(q, k, v, o=o, lse=lse, causal=w.causal, window_left=w.window_left)
@@ -395,37 +484,54 @@ def run_ours(args, world, rank, local):
         ea.attn_bwd(q, k, v, o, lse, dout, causal=w.causal, window_left=w.window_left,
                     dq=dq_t, dk=dk_t, dv=dv_t, workspace=bws)
 
-    btimes, blaunches = timed_kernel_loop(bwd, args.steps, args.warmup, world, flush, None)
-    bms = statistics.mean(btimes)
-    bms_max = max_over_ranks(bms, world)
+    btimes, blaunches = timed_kernel_loop(bwd, args.steps, args.warmup, world, flush)
+    bst = time_stats(btimes)
+    bms_max = max_over_ranks(bst["mean"], world)
     b_flops = 2.5 * flops
-    b_value = whole_job_rate(b_flops, bms_max, world) / 1e12
-    b_achieved = b_flops / (bms * 1e-3) / 1e12
+    backward = {
+        "workload": f"{w.name}, backward (dQ, dK, dV)",
+        "value": whole_job_rate(b_flops, bms_max, world) / 1e12, "unit": "TFLOP/s",
+        "ms_per_step": bms_max, "ms": bst,
+        "flop_count": "2.5 x the forward's mask-adjusted FLOPs",
+        "roofline": dict(tensor_roofline(b_flops / (bst["mean"] * 1e-3) / 1e12, peaks, peak_src,
+                                         "bwd_prep_kernel + bwd_main_kernel<128> + bwd_finalize_kernel",
+                                         recorded_traffic("bwd_main_kernel", args.workload, resized)),
+                         traffic_kernel="bwd_main_kernel<128>"),
+        "gpu_launches": blaunches,
+    }
     del dout, dq_t, dk_t, dv_t, bws
 
-    # merge leg (sequence-sharded attention's combine): 4 fp32 parts of the
-    # prefill output shape -> bf16 O and LSE; HBM-bound, inputs far above L2
+    # ---- merge leg (sequence-sharded attention's combine): 4 fp32 parts of the
+    # MHA N=2048 output shape -> bf16 O and LSE; HBM-bound, inputs far above L2
+    mw = ai.MHA_2K
     R_m = 4
     g_m = torch.Generator(device="cpu")
     g_m.manual_seed(shard_seed(rank) + 31)
-    mo_parts = torch.randn((R_m, w.B, w.Nq, w.Hq, w.d), generator=g_m).to(dev)
-    ml_parts = torch.randn((R_m, w.B, w.Hq, w.Nq), generator=g_m).to(dev)
-    m_out = torch.empty((w.B, w.Nq, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
-    m_lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=dev)
+    mo_parts = torch.randn((R_m, mw.B, mw.Nq, mw.Hq, mw.d), generator=g_m).to(dev)
+    ml_parts = torch.randn((R_m, mw.B, mw.Hq, mw.Nq), generator=g_m).to(dev)
+    m_out = torch.empty((mw.B, mw.Nq, mw.Hq, mw.d), dtype=torch.bfloat16, device=dev)
+    m_lse = torch.empty((mw.B, mw.Hq, mw.Nq), dtype=torch.float32, device=dev)
 
     def merge():
         ea.attn_merge(mo_parts, ml_parts, o=m_out, lse=m_lse)
 
-    mtimes, mlaunches = timed_kernel_loop(merge, args.steps, args.warmup, world, None, None)
-    mms = statistics.mean(mtimes)
-    mms_max = max_over_ranks(mms, world)
-    m_rows = w.B * w.Nq * w.Hq
-    m_bytes = R_m * m_rows * (w.d + 1) * 4 + m_rows * (w.d * 2 + 4)
-    m_value = whole_job_rate(m_bytes, mms_max, world) / 1e9
-    m_achieved = m_bytes / (mms * 1e-3) / 1e9
+    mtimes, mlaunches = timed_kernel_loop(merge, args.steps, args.warmup, world, None)
+    mst = time_stats(mtimes)
+    mms_max = max_over_ranks(mst["mean"], world)
+    m_rows = mw.B * mw.Nq * mw.Hq
+    m_bytes = R_m * m_rows * (mw.d + 1) * 4 + m_rows * (mw.d * 2 + 4)
+    merge_leg = {
+        "workload": f"merge of {R_m} fp32 parts, {mw.name} output shape",
+        "value": whole_job_rate(m_bytes, mms_max, world) / 1e9, "unit": "GB/s",
+        "ms_per_step": mms_max, "ms": mst,
+        "roofline": hbm_roofline(m_bytes / (mst["mean"] * 1e-3) / 1e9, peaks, peak_src,
+                                 "attn_merge_kernel<128>", recorded_traffic("merge", "merge4"),
+                                 m_bytes),
+        "gpu_launches": mlaunches,
+    }
     del mo_parts, ml_parts, m_out, m_lse
 
-    # packed variable-length prefill leg: 16 causal sequences with seeded
+    # ---- packed variable-length prefill leg: 16 causal sequences with seeded
     # lengths in [256, 4096], MHA H32 d128, no padding
     vl_lens = ai.varlen_lengths(16, 256, 4096, seed=shard_seed(rank) + 13)
     vq_h, vk_h, vv_h, vcq_h, vck_h = ai.make_varlen(vl_lens, vl_lens, 32, 32, 128,
@@ -438,15 +544,23 @@ def run_ours(args, world, rank, local):
     def fwd_varlen():
         ea.attn_fwd_varlen(vq, vk, vv, vcq, vck, vmax, vmax, o=vo, lse=vlse, causal=True)
 
-    vtimes, vlaunches = timed_kernel_loop(fwd_varlen, args.steps, args.warmup, world, flush, None)
-    vms = statistics.mean(vtimes)
-    vms_max = max_over_ranks(vms, world)
+    vtimes, vlaunches = timed_kernel_loop(fwd_varlen, args.steps, args.warmup, world, flush)
+    vst = time_stats(vtimes)
+    vms_max = max_over_ranks(vst["mean"], world)
     v_flops = sum(metrics.attn_flops(1, 32, n, n, 128, True, -1) for n in vl_lens)
-    v_value = whole_job_rate(v_flops, vms_max, world) / 1e12
-    v_achieved = v_flops / (vms * 1e-3) / 1e12
+    varlen = {
+        "workload": f"MHA causal packed prefill, 16 sequences of {min(vl_lens)}-{max(vl_lens)} "
+                    f"tokens ({sum(vl_lens)} total) H32 d128",
+        "value": whole_job_rate(v_flops, vms_max, world) / 1e12, "unit": "TFLOP/s",
+        "ms_per_step": vms_max, "ms": vst,
+        "roofline": tensor_roofline(v_flops / (vst["mean"] * 1e-3) / 1e12, peaks, peak_src,
+                                    "attn_fwd_kernel<128,false> (packed)",
+                                    recorded_traffic("attn_fwd_kernel", "varlen")),
+        "gpu_launches": vlaunches,
+    }
     del vq, vk, vv, vo
 
-    # decode leg
+    # ---- decode leg
     dw = ai.GQA_DECODE
     if args.decode_batch:
         dw = dataclasses.replace(dw, B=args.decode_batch, name=f"{dw.name} [batch {args.decode_batch}]")
@@ -461,15 +575,23 @@ def run_ours(args, world, rank, local):
         ea.attn_decode(qd, kc, vc, o=od, lse=lsed, num_splits=args.decode_splits, workspace=ws)
 
     # the cache (2.1 GB) is far larger than L2, so no flush between decode steps
-    dtimes, dlaunches = timed_kernel_loop(dec, args.steps, args.warmup, world, None, None)
-    dms = statistics.mean(dtimes)
-    dms_max = max_over_ranks(dms, world)
+    dtimes, dlaunches = timed_kernel_loop(dec, args.steps, args.warmup, world, None)
+    dst = time_stats(dtimes)
+    dms_max = max_over_ranks(dst["mean"], world)
     kv_bytes = metrics.decode_kv_bytes([dw.Nk] * dw.B, dw.Hkv, dw.d)
     d_all = metrics.decode_bytes(dw.B, dw.Hq, dw.Hkv, [dw.Nk] * dw.B, dw.d)
-    d_value = whole_job_rate(kv_bytes, dms_max, world) / 1e9
+    decode = {
+        "workload": dw.name, "value": whole_job_rate(kv_bytes, dms_max, world) / 1e9,
+        "unit": "GB/s", "ms_per_step": dms_max, "ms": dst,
+        "roofline": hbm_roofline(kv_bytes / (dst["mean"] * 1e-3) / 1e9, peaks, peak_src,
+                                 "decode_split_kernel<128,4> + decode_combine_kernel<128>",
+                                 recorded_traffic("decode", "decode", bool(args.decode_batch)),
+                                 d_all),
+        "gpu_launches": dlaunches,
+    }
 
-    # paged decode leg: the same logical cache scattered into shuffled pages of
-    # args.page_size keys (a seeded permutation; unused pool pages are never read)
+    # ---- paged decode leg: the same logical cache scattered into shuffled pages
+    # of args.page_size keys (a seeded permutation; unused pool pages are never read)
     ps = args.page_size
     per_seq = dw.Nk // ps
     n_pages = dw.B * per_seq + 64
@@ -487,13 +609,24 @@ def run_ours(args, world, rank, local):
         ea.attn_decode_paged(qd, kpg, vpg, bt, o=od, lse=lsed, num_splits=args.decode_splits,
                              workspace=ws)
 
-    ptimes, plaunches = timed_kernel_loop(dec_paged, args.steps, args.warmup, world, None, None)
-    pms = statistics.mean(ptimes)
-    pms_max = max_over_ranks(pms, world)
-    p_value = whole_job_rate(kv_bytes, pms_max, world) / 1e9
+    ptimes, plaunches = timed_kernel_loop(dec_paged, args.steps, args.warmup, world, None)
+    pst = time_stats(ptimes)
+    pms_max = max_over_ranks(pst["mean"], world)
+    decode_paged = {
+        "workload": f"{dw.name}, paged cache ({ps}-key pages, shuffled pool)", "page_size": ps,
+        "value": whole_job_rate(kv_bytes, pms_max, world) / 1e9, "unit": "GB/s",
+        "ms_per_step": pms_max, "ms": pst,
+        "roofline": hbm_roofline(kv_bytes / (pst["mean"] * 1e-3) / 1e9, peaks, peak_src,
+                                 "decode_split_kernel<128,4,paged> + decode_combine_kernel<128>",
+                                 recorded_traffic("decode_paged", f"decode_p{ps}",
+                                                  bool(args.decode_batch)),
+                                 d_all),
+        "gpu_launches": plaunches,
+    }
     del kpg, vpg
+    sampler.stop()
 
-    # end-to-end through the public API with host buffers
+    # ---- end-to-end through the public API with host buffers (headline workload)
     e2e = None
     if not args.no_e2e:
         qp, kp, vp = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
@@ -514,21 +647,28 @@ def run_ours(args, world, rank, local):
         e2e = {"value": whole_job_rate(flops, e_ms, world) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
 
+    # ---- the oracle on the host cores: the headline workload, and the GQA
+    # sliding-window workload once
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline_block(w, q_h, k_h, v_h)
+        cpu = cpu_baseline_block(w, q_h, k_h, v_h, budget_s=12.0)
+        for leg in legs:
+            if leg["key"] == "gqa32k":
+                gw = ai.GQA_SWA_32K
+                gq, gk, gv = ai.make_for(gw, seed=shard_seed(rank))
+                leg["cpu_baseline"] = cpu_baseline_block(gw, gq, gk, gv, budget_s=6.0)
+                del gq, gk, gv
 
     if rank != 0:
         return
-    peak_t = peaks["bf16_tflops"]
     line = {
         "metric": METRIC,
-        "value": value,
+        "value": head["value"],
         "unit": "TFLOP/s",
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": ms_max,
+        "ms_per_step": head["ms_per_step"],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -537,71 +677,20 @@ def run_ours(args, world, rank, local):
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "seq_len": w.Nq,
                    "d": w.d, "causal": w.causal, "window_left": w.window_left,
                    "parallelism": f"independent batch per GPU x{world}",
-                   "l2": "256 MiB memset flush before every timed step (outside the events)",
+                   "l2": "256 MiB memset flush before every timed prefill/backward step "
+                         "(outside the events); decode and merge inputs exceed L2",
                    "flop_count": "4*d*allowed (i,j) pairs (mask-adjusted)"},
-        "pct_bf16_peak": 100.0 * achieved / peak_t,
-        "tile_tflops": tiles * 4.0 * 128 * 128 * w.d / (ms * 1e-3) / 1e12,
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
-                     "frac": achieved / peak_t, "peak_source": f"{peak_src} bf16_tflops (burst)",
-                     "kernel": "attn_fwd_kernel<128,false>",
-                     "traffic": recorded_traffic("attn_fwd_kernel", args.workload, bool(args.batch)),
-                     "algorithmic_bytes": metrics.attn_fwd_bytes(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d)},
-        "decode": {
-            "workload": dw.name, "value": d_value, "unit": "GB/s", "ms_per_step": dms_max,
-            "roofline": {"bound": "hbm", "achieved": kv_bytes / (dms * 1e-3) / 1e9,
-                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": kv_bytes / (dms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                         "peak_source": f"{peak_src} hbm_gbs",
-                         "kernel": "decode_split_kernel<128,4> + decode_combine_kernel<128>",
-                         "algorithmic_bytes": d_all,
-                         "traffic": recorded_traffic("decode", "decode", bool(args.decode_batch))},
-            "gpu_launches": dlaunches,
-        },
-        "backward": {
-            "workload": f"{w.name}, backward (dQ, dK, dV)", "value": b_value, "unit": "TFLOP/s",
-            "ms_per_step": bms_max,
-            "flop_count": "2.5 x the forward's mask-adjusted FLOPs",
-            "roofline": {"bound": "tensor", "achieved": b_achieved, "peak": peak_t,
-                         "unit": "TFLOP/s", "frac": b_achieved / peak_t,
-                         "peak_source": f"{peak_src} bf16_tflops (burst)",
-                         "kernel": "bwd_prep_kernel + bwd_main_kernel<128> + bwd_finalize_kernel",
-                         "traffic": recorded_traffic("bwd_main_kernel", args.workload, bool(args.batch)),
-                         "traffic_kernel": "bwd_main_kernel<128>"},
-            "gpu_launches": blaunches,
-        },
-        "merge": {
-            "workload": f"merge of {R_m} fp32 parts, {w.name} output shape", "value": m_value,
-            "unit": "GB/s", "ms_per_step": mms_max,
-            "roofline": {"bound": "hbm", "achieved": m_achieved, "peak": peaks["hbm_gbs"],
-                         "unit": "GB/s", "frac": m_achieved / peaks["hbm_gbs"],
-                         "peak_source": f"{peak_src} hbm_gbs", "kernel": "attn_merge_kernel<128>",
-                         "algorithmic_bytes": m_bytes, "traffic": None},
-            "gpu_launches": mlaunches,
-        },
-        "varlen": {
-            "workload": f"MHA causal packed prefill, 16 sequences of {min(vl_lens)}-{max(vl_lens)} "
-                        f"tokens ({sum(vl_lens)} total) H32 d128",
-            "value": v_value, "unit": "TFLOP/s", "ms_per_step": vms_max,
-            "roofline": {"bound": "tensor", "achieved": v_achieved, "peak": peak_t,
-                         "unit": "TFLOP/s", "frac": v_achieved / peak_t,
-                         "peak_source": f"{peak_src} bf16_tflops (burst)",
-                         "kernel": "attn_fwd_kernel<128,false> (packed)",
-                         "traffic": recorded_traffic("attn_fwd_kernel", "varlen")},
-            "gpu_launches": vlaunches,
-        },
-        "decode_paged": {
-            "workload": f"{dw.name}, paged cache ({ps}-key pages, shuffled pool)", "page_size": ps,
-            "value": p_value, "unit": "GB/s", "ms_per_step": pms_max,
-            "roofline": {"bound": "hbm", "achieved": kv_bytes / (pms * 1e-3) / 1e9,
-                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": kv_bytes / (pms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                         "peak_source": f"{peak_src} hbm_gbs",
-                         "kernel": "decode_split_kernel<128,4,paged> + decode_combine_kernel<128>",
-                         "algorithmic_bytes": d_all,
-                         "traffic": recorded_traffic("decode_paged", f"decode_p{ps}", bool(args.decode_batch))},
-            "gpu_launches": plaunches,
-        },
-        "clocks": clocks,
+        "ms": head["ms"],
+        "pct_bf16_peak": head["pct_bf16_peak"],
+        "tile_tflops": head["tile_tflops"],
+        "roofline": head["roofline"],
+        "prefill_legs": legs,
+        "decode": decode,
+        "backward": backward,
+        "merge": merge_leg,
+        "varlen": varlen,
+        "decode_paged": decode_paged,
+        "clocks": sampler.summary(),
         "gpu_launches": launches,
         "e2e": e2e,
         "cpu_baseline": cpu,

@@ -17,29 +17,29 @@
 //                       accumulator with vector atomics
 //   bwd_finalize_kernel dQ accumulator -> bf16
 //
-// bwd_main_kernel warp roles (320 threads):
-//   warps 0-3  elementwise, thread = TMEM lane = key row: P, dS per block; at
-//              the end dK, dV
+// bwd_main_kernel warp roles (352 threads):
+//   warps 0-3  elementwise, thread = TMEM lane = key row: P, then dS, per
+//              block; at the end dK, dV
 //   warps 4-7  dQ, thread = TMEM lane = query row: read dQ_i out of tensor
-//              memory, add it to the accumulator; stage the next block's
-//              lse2 / delta values in shared memory
+//              memory, add it to the accumulator
 //   warp 8     tensor-core issuer (whole warp, one elected lane issues)
 //   warp 9     TMA producer (one lane): K_j, V_j once; Q_i, dO_i per block
 //              through a 2-stage ring (the next block's tiles load during this one)
-// Per query block (tile = 128 x 128):
-//   Sᵀ  = K_j Q_iᵀ        SS, both K-major, two 64-query halves -> TMEM cols [0,128)
-//   dPᵀ = V_j dO_iᵀ       SS, both K-major, two 64-query halves -> TMEM cols [128,256)
-//   elementwise: Pᵀ = exp2(Sᵀ c - lse2), dSᵀ = Pᵀ (dPᵀ - delta); Pᵀ and dSᵀ
-//     as bf16 pairs over cols [0,64) and [128,192); dSᵀ also to shared memory
+//   warp 10    stages each block's lse2 / delta values in shared memory
+// Per query block (tile = 128 x 128), TMEM cols [0,128) Sᵀ / Pᵀ, [128,256)
+// dPᵀ / dQ_i, [256,256+D) dV, [256+D,256+2D) dK:
+//   Sᵀ  = K_j Q_iᵀ        SS, both K-major (N = 128)
+//   phase P: Pᵀ = exp2(Sᵀ c - lse2) as bf16 pairs over cols [0,64); the pairs
+//     stay in registers
 //   dV += Pᵀ dO_i         TS: A = Pᵀ (TMEM), B = dO_i MN-major
-//   dK += dSᵀ Q_i         TS: A = dSᵀ (TMEM), B = Q_i MN-major
+//   dPᵀ = V_j dO_iᵀ       SS, both K-major (N = 128)
+//   phase dS: dSᵀ = Pᵀ (dPᵀ - delta) from those bf16 P, to shared memory only
 //   dQ_i = dS K_j         SS: A = dS MN-major (the dSᵀ tile read transposed),
-//                         B = K_j MN-major; 64 columns of d at a time into the
-//                         free cols [64,128) and [192,256)
-// The first half of the next block's Sᵀ and dPᵀ goes into cols [0,64) and
-// [128,192) as soon as dV and dK are done with them, so the elementwise warps
-// start on it while the dQ warps still read dQ_i out of cols [64,128) and
-// [192,256); the second half follows once that read-out is done.
+//                         B = K_j MN-major (N = D), into the dPᵀ columns
+//   dK += dSᵀ Q_i         SS: A = the dSᵀ tile K-major, B = Q_i MN-major
+// The next block's Sᵀ goes in as soon as dV has read Pᵀ, so the elementwise
+// warps find it ready after their dS phase; the next dPᵀ follows the
+// read-out of dQ_i.
 // All waits are bounded (sm100_ptx.cuh).
 #pragma once
 
@@ -66,31 +66,42 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
       : "memory");
 }
 
-// Pᵀ and dSᵀ of one key row over 32 queries [c0, c0 + 32) of the block, as
-// bf16 pairs: P = exp2(S c2 - lse2), dS = P (dP - delta). MASK: only the
-// queries in [c_lo, c_hi] are allowed, the rest get P = 0.
+// Pᵀ of one key row over 32 queries [c0, c0 + 32) of the block, as bf16 pairs:
+// P = exp2(S c2 - lse2). MASK: only the queries in [c_lo, c_hi] are allowed,
+// the rest get P = 0.
 template <bool MASK>
-__device__ __forceinline__ void bwd_p_ds(const uint32_t* sr, const uint32_t* dr, const float* lsr,
-                                         const float* dlt, int c0, int c_lo, int c_hi, float c2,
-                                         uint32_t* pw, uint32_t* dw) {
+__device__ __forceinline__ void bwd_p(const uint32_t* sr, const float* lsr, int c0, int c_lo, int c_hi,
+                                      float c2, uint32_t* pw) {
   const float4* l4 = reinterpret_cast<const float4*>(lsr + c0);
-  const float4* d4 = reinterpret_cast<const float4*>(dlt + c0);
 #pragma unroll
   for (int e = 0; e < 32; e += 4) {
-    const float4 lv = l4[e / 4], dv = d4[e / 4];
-    const float l[4] = {lv.x, lv.y, lv.z, lv.w}, d[4] = {dv.x, dv.y, dv.z, dv.w};
-    float pp[4], ds[4];
+    const float4 lv = l4[e / 4];
+    const float l[4] = {lv.x, lv.y, lv.z, lv.w};
+    float pp[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const float x = fmaf(__uint_as_float(sr[e + u]), c2, -l[u]);
-      pp[u] = ex2_approx(x);
+      pp[u] = ex2_approx(fmaf(__uint_as_float(sr[e + u]), c2, -l[u]));
       if (MASK) pp[u] = (c0 + e + u >= c_lo && c0 + e + u <= c_hi) ? pp[u] : 0.f;
-      ds[u] = pp[u] * (__uint_as_float(dr[e + u]) - d[u]);
     }
     pw[e / 2] = pack_bf16x2(pp[0], pp[1]);
     pw[e / 2 + 1] = pack_bf16x2(pp[2], pp[3]);
-    dw[e / 2] = pack_bf16x2(ds[0], ds[1]);
-    dw[e / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
+  }
+}
+
+// dSᵀ = Pᵀ (dPᵀ - delta) of one key row over 32 queries [c0, c0 + 32), from the
+// bf16 pairs of Pᵀ (the values the dV product uses), as bf16 pairs.
+__device__ __forceinline__ void bwd_ds(const uint32_t* dr, const uint32_t* pw, const float* dlt, int c0,
+                                       uint32_t* dw) {
+  const float4* d4 = reinterpret_cast<const float4*>(dlt + c0);
+#pragma unroll
+  for (int e = 0; e < 32; e += 4) {
+    const float4 dv = d4[e / 4];
+    const float ds0 = bf16lo(pw[e / 2]) * (__uint_as_float(dr[e]) - dv.x);
+    const float ds1 = bf16hi(pw[e / 2]) * (__uint_as_float(dr[e + 1]) - dv.y);
+    const float ds2 = bf16lo(pw[e / 2 + 1]) * (__uint_as_float(dr[e + 2]) - dv.z);
+    const float ds3 = bf16hi(pw[e / 2 + 1]) * (__uint_as_float(dr[e + 3]) - dv.w);
+    dw[e / 2] = pack_bf16x2(ds0, ds1);
+    dw[e / 2 + 1] = pack_bf16x2(ds2, ds3);
   }
 }
 
@@ -190,26 +201,27 @@ struct BwdLayout {
   static constexpr int B_KV = 0;     // K_j, V_j loaded
   static constexpr int B_QD = 1;     // Q_i, dO_i loaded, + stage
   static constexpr int B_QDE = 3;    // Q_i, dO_i stage free again, + stage
-  static constexpr int B_SD0 = 5;    // Sᵀ and dPᵀ of queries [0, 64) in TMEM
-  static constexpr int B_PR = 6;     // Pᵀ, dSᵀ written (128 arrivals)
-  static constexpr int B_QR = 7;     // dQ_i in TMEM
-  static constexpr int B_QF = 8;     // dQ_i read out (128 dQ-warp arrivals)
-  static constexpr int B_DONE = 9;   // every dK / dV product complete
-  static constexpr int B_LD = 10;    // block lse2 / delta values in shared memory (128 dQ-warp arrivals)
-  static constexpr int B_SD1 = 11;   // Sᵀ and dPᵀ of queries [64, 128) in TMEM
-  static constexpr int B_KVD = 12;   // dV, dK products of the block complete (issuer only)
-  static constexpr int NBAR = 13;
+  static constexpr int B_SS = 5;     // Sᵀ in TMEM
+  static constexpr int B_SP = 6;     // dPᵀ in TMEM (and the previous dQ product done)
+  static constexpr int B_PA = 7;     // Pᵀ written (128 elementwise arrivals)
+  static constexpr int B_PB = 8;     // dSᵀ written to shared memory (128 arrivals)
+  static constexpr int B_DVD = 9;    // dV product of the block complete (issuer only)
+  static constexpr int B_QR = 10;    // dQ_i in TMEM
+  static constexpr int B_QF = 11;    // dQ_i read out (128 dQ-warp arrivals)
+  static constexpr int B_DONE = 12;  // every dK / dV product complete
+  static constexpr int B_LD = 13;    // block lse2 / delta values in shared memory (32 arrivals)
+  static constexpr int NBAR = 14;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;      // [0] TMEM base, [1] abort flag
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = BYTES + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_ST = 0, COL_DPT = 128, COL_DV = 256, COL_DK = 256 + D;
-  static constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64, 0);      // one 64-query half
+  static constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, 0);
   static constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, D, 1);
-  static constexpr uint32_t IDESC_DQ = idesc_bf16_f32_amn(128, 64, 1);
+  static constexpr uint32_t IDESC_DQ = idesc_bf16_f32_amn(128, D, 1);
 };
 
-constexpr int kBwdThreads = 320;
+constexpr int kBwdThreads = 352;
 
 // Query blocks that hold at least one allowed (query, key) pair with a key in
 // [kb0, kb1]: [i_lo, i_hi], empty when i_hi < i_lo.
@@ -263,14 +275,15 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       mbar_init(bar(L::B_QD + st), 1);
       mbar_init(bar(L::B_QDE + st), 1);
     }
-    mbar_init(bar(L::B_SD0), 1);
-    mbar_init(bar(L::B_SD1), 1);
-    mbar_init(bar(L::B_KVD), 1);
-    mbar_init(bar(L::B_PR), 128);
+    mbar_init(bar(L::B_SS), 1);
+    mbar_init(bar(L::B_SP), 1);
+    mbar_init(bar(L::B_PA), 128);
+    mbar_init(bar(L::B_PB), 128);
+    mbar_init(bar(L::B_DVD), 1);
     mbar_init(bar(L::B_QR), 1);
     mbar_init(bar(L::B_QF), 128);
     mbar_init(bar(L::B_DONE), 1);
-    mbar_init(bar(L::B_LD), 128);
+    mbar_init(bar(L::B_LD), 32);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -296,9 +309,9 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     bool ok = true;
     for (int n = 0; ok && n < total; ++n) {
       const int i = i_lo + n % nblk;
-      const int par = n & 1;
-      if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_SD0), uint32_t(par), abort_flag)))) break;
-      if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_LD), uint32_t(par), abort_flag)))) break;
+      const uint32_t par = uint32_t(n & 1);
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_SS), par, abort_flag)))) break;
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_LD), par, abort_flag)))) break;
       tc_fence_after();
       // allowed queries of this key within the block: [c_lo, c_hi]
       const int q0 = i * 128;
@@ -306,26 +319,35 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       if (key >= p.Nk) c_hi = -1;
       if (p.causal) c_lo = max(c_lo, key - off - q0);                    // key <= q + off
       if (p.window_left >= 0) c_hi = min(c_hi, key + p.window_left - off - q0);
-      // 32 queries at a time: read their Sᵀ and dPᵀ columns, then write the
-      // bf16 pairs of Pᵀ and dSᵀ over columns already read (chunk c of 32
-      // queries -> columns [16c, 16c + 16))
+      // phase A, 32 queries at a time: Pᵀ over columns of Sᵀ already read
+      // (chunk c -> columns [16c, 16c + 16)); the bf16 pairs stay in registers
+      uint32_t pw[4][16];
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         const int c0 = 32 * cc;
-        if (cc == 2) {                                       // second 64-query half
-          if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_SD1), uint32_t(par), abort_flag)))) break;
-          tc_fence_after();
-        }
-        uint32_t sr[32], dr[32], pw[16], dw[16];
+        uint32_t sr[32];
         tmem_ld32(tST + c0, sr);
-        tmem_ld32(tDPT + c0, dr);
         tmem_wait_ld();
         if (__all_sync(0xffffffffu, c_lo <= c0 && c_hi >= c0 + 31))
-          bwd_p_ds<false>(sr, dr, lsr, dlt, c0, c_lo, c_hi, c2, pw, dw);
+          bwd_p<false>(sr, lsr, c0, c_lo, c_hi, c2, pw[cc]);
         else
-          bwd_p_ds<true>(sr, dr, lsr, dlt, c0, c_lo, c_hi, c2, pw, dw);
-        tmem_st16(tST + 16 * cc, pw);
-        tmem_st16(tDPT + 16 * cc, dw);
+          bwd_p<true>(sr, lsr, c0, c_lo, c_hi, c2, pw[cc]);
+        tmem_st16(tST + 16 * cc, pw[cc]);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(L::B_PA));
+      // phase B: dSᵀ once dPᵀ is in TMEM. B_SP also covers the previous dQ
+      // product, the last reader of the dS tile in shared memory.
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_SP), par, abort_flag)))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        const int c0 = 32 * cc;
+        uint32_t dr[32], dw[16];
+        tmem_ld32(tDPT + c0, dr);
+        tmem_wait_ld();
+        bwd_ds(dr, pw[cc], dlt, c0, dw);
         // dSᵀ row of this key -> shared memory block cc / 2 (queries 64h..64h+63),
         // 16-byte chunks swizzled by (row & 7)
 #pragma unroll
@@ -337,11 +359,9 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                        "r"(dw[4 * ch + 3]) : "memory");
         }
       }
-      if (!ok) break;
-      tmem_wait_st();
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       tc_fence_before();
-      mbar_arrive(bar(L::B_PR));
+      mbar_arrive(bar(L::B_PB));
     }
     // ---- dK, dV of this key row ---------------------------------------------
     const bool have = ok && total > 0 &&
@@ -380,45 +400,15 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   } else if (warp < 8) {
     // ======================= dQ warps ========================================
     const int r = int(threadIdx.x) - 128;                    // TMEM lane = query row in the block
-    const uint32_t lane_off = uint32_t((warp - 4) * 32) << 16;
-    float* lse2_s = reinterpret_cast<float*>(smem + L::OFF_LD);
-    float* delta_s = lse2_s + 128;
-    // lse2 (log2 units, 0 for empty rows) and delta of query row r of block n
-    auto row_values = [&](int n, float& l2, float& dl) {
-      const int hq = hkv * G + n / nblk, q = (i_lo + n % nblk) * 128 + r;
-      const bool qv = q < p.Nq;
-      const float l = qv ? __ldg(p.lse + (size_t(b) * p.Hq + hq) * p.Nq + q) : 0.f;
-      l2 = (qv && l > -CUDART_INF_F) ? l * 1.4426950408889634f : 0.f;
-      dl = qv ? __ldg(p.delta + (size_t(b) * p.Hq + hq) * p.Nq + q) : 0.f;
-    };
-    if (total > 0) {
-      float l2, dl;
-      row_values(0, l2, dl);
-      lse2_s[r] = l2;
-      delta_s[r] = dl;
-      mbar_arrive(bar(L::B_LD));
-    }
+    const uint32_t tDQ = tmem + (uint32_t((warp - 4) * 32) << 16) + L::COL_DPT;
     for (int n = 0; n < total; ++n) {
       const int hq = hkv * G + n / nblk, q = (i_lo + n % nblk) * 128 + r;
-      float l2 = 0.f, dl = 0.f;
-      if (n + 1 < total) row_values(n + 1, l2, dl);
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_QR), uint32_t(n & 1), abort_flag))) break;
+      const uint32_t par = uint32_t(n & 1);
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_QR), par, abort_flag))) break;
       tc_fence_after();
-      // one buffer is enough: B_QR(n) completes after the products issued once
-      // every elementwise thread arrived on B_PR(n), i.e. after every read of
-      // block n's values
-      if (n + 1 < total) {
-        lse2_s[r] = l2;
-        delta_s[r] = dl;
-        mbar_arrive(bar(L::B_LD));
-      }
       uint32_t qr[D];
 #pragma unroll
-      for (int h = 0; h < D / 64; ++h) {
-        const uint32_t col = tmem + lane_off + (h == 0 ? L::COL_ST : L::COL_DPT) + 64;
-        tmem_ld32(col, qr + 64 * h);
-        tmem_ld32(col + 32, qr + 64 * h + 32);
-      }
+      for (int c = 0; c < D / 32; ++c) tmem_ld32(tDQ + 32 * c, qr + 32 * c);
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(bar(L::B_QF));
@@ -447,76 +437,73 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const uint64_t dQ_mn = smem_desc_sw128(sb + L::OFF_Q, L::HALF, 1024);
     const uint64_t dO_mn = smem_desc_sw128(sb + L::OFF_DO, L::HALF, 1024);
     const uint64_t dS_mn = smem_desc_sw128(sb + L::OFF_DS, L::HALF, 1024);
+    const uint64_t dS_k = smem_desc_sw128(sb + L::OFF_DS, 16, 1024);
     const uint64_t dKj_mn = smem_desc_sw128(sb + L::OFF_K, L::HALF, 1024);
     const uint32_t tST = tmem + L::COL_ST, tDPT = tmem + L::COL_DPT;
     const uint32_t tDV = tmem + L::COL_DV, tDK = tmem + L::COL_DK;
-    // Sᵀ = K_j Q_iᵀ and dPᵀ = V_j dO_iᵀ (K = d) for queries [64h, 64h + 64) of
-    // block n: TMEM cols [64h, 64h + 64) of each
-    auto issue_sdp = [&](int n, int h) {
-      const uint32_t so = uint32_t(((n & 1) * L::TILE + h * 64 * 128) >> 4);
+    // A_j X_iᵀ (K = d) into TMEM cols [col, col + 128): Sᵀ (A = K, X = Q) or
+    // dPᵀ (A = V, X = dO) of block n
+    auto issue_rows = [&](uint32_t dst, uint64_t a_k, uint64_t x_k, int n) {
+      const uint32_t so = uint32_t(((n & 1) * L::TILE) >> 4);
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
         const uint32_t o = ((k / 4) * L::HALF + (k % 4) * 32) >> 4;
-        if (elect_one()) mma_ss(tST + 64 * h, dK_k + o, dQ_k + so + o, L::IDESC_S, k > 0 ? 1u : 0u);
-      }
-#pragma unroll
-      for (int k = 0; k < D / 16; ++k) {
-        const uint32_t o = ((k / 4) * L::HALF + (k % 4) * 32) >> 4;
-        if (elect_one()) mma_ss(tDPT + 64 * h, dV_k + o, dO_k + so + o, L::IDESC_S, k > 0 ? 1u : 0u);
+        if (elect_one()) mma_ss(dst, a_k + o, x_k + so + o, L::IDESC_S, k > 0 ? 1u : 0u);
       }
     };
     bool alive = total > 0 && wwait(L::B_KV, 0u) && wwait(L::B_QD, 0u);
     if (alive) {
       tc_fence_after();
-      issue_sdp(0, 0);
-      commit(L::B_SD0);
+      issue_rows(tST, dK_k, dQ_k, 0);
+      commit(L::B_SS);
     }
     for (int n = 0; alive && n < total; ++n) {
       const uint32_t par = uint32_t(n & 1);
       const int stg = n & 1;                                     // Q/dO stage of this block
       const uint32_t so = uint32_t(stg * (L::TILE >> 4));       // its descriptor offset
-      // second half once dQ of the previous block (cols [64, 128)) is read out
+      const bool next = n + 1 < total;
+      // dPᵀ once dQ of the previous block (cols [128, 128 + D)) is read out;
+      // the commit also covers that dQ product, the last reader of the dS tile
       if (n > 0 && !(alive = wwait(L::B_QF, par ^ 1u))) break;
       tc_fence_after();
-      issue_sdp(n, 1);
-      commit(L::B_SD1);
-      if (!(alive = wwait(L::B_PR, par))) break;
+      issue_rows(tDPT, dV_k, dO_k, n);
+      commit(L::B_SP);
+      // dV += Pᵀ dO_i (K = 128 queries, 16 per MMA) once Pᵀ is in TMEM
+      if (!(alive = wwait(L::B_PA, par))) break;
       tc_fence_after();
-      // dV += Pᵀ dO_i, dK += dSᵀ Q_i (K = 128 queries, 16 per MMA)
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
         const uint32_t o = (k * 16 * 128) >> 4;
         if (elect_one()) mma_ts(tDV, tST + 8 * k, dO_mn + so + o, L::IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
       }
+      if (next) {
+        // Sᵀ of the next block over cols [0, 128): Pᵀ (cols [0, 64)) must have
+        // been read by the dV product, and the elementwise warps are done with Sᵀ
+        commit(L::B_DVD);
+        if (!(alive = wwait(L::B_QD + ((n + 1) & 1), uint32_t(((n + 1) >> 1) & 1)))) break;
+        if (!(alive = wwait(L::B_DVD, par))) break;
+        tc_fence_after();
+        issue_rows(tST, dK_k, dQ_k, n + 1);
+        commit(L::B_SS);
+      }
+      // once dSᵀ is in shared memory: dQ_i = dS K_j (K = 128 keys) into the dPᵀ
+      // columns, already read, then dK += dSᵀ Q_i with dSᵀ read K-major from the
+      // same tile (K = 128 queries, 16 per MMA)
+      if (!(alive = wwait(L::B_PB, par))) break;
+      tc_fence_after();
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
         const uint32_t o = (k * 16 * 128) >> 4;
-        if (elect_one()) mma_ts(tDK, tDPT + 8 * k, dQ_mn + so + o, L::IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
-      }
-      const bool next = n + 1 < total;
-      if (next) commit(L::B_KVD);
-      // dQ_i = dS K_j, 64 columns of d at a time (K = 128 keys)
-#pragma unroll
-      for (int h = 0; h < D / 64; ++h) {
-        const uint32_t dst = (h == 0 ? tST : tDPT) + 64;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint32_t o = (k * 16 * 128) >> 4;
-          if (elect_one())
-            mma_ss(dst, dS_mn + o, dKj_mn + ((h * L::HALF) >> 4) + o, L::IDESC_DQ, k > 0 ? 1u : 0u);
-        }
+        if (elect_one()) mma_ss(tDPT, dS_mn + o, dKj_mn + o, L::IDESC_DQ, k > 0 ? 1u : 0u);
       }
       commit(L::B_QR);
-      commit(L::B_QDE + stg);
-      if (next) {
-        // first half of the next block: its columns [0, 64) held Pᵀ and dSᵀ,
-        // free once the dV and dK products finished reading them
-        if (!(alive = wwait(L::B_QD + ((n + 1) & 1), uint32_t(((n + 1) >> 1) & 1)))) break;
-        if (!(alive = wwait(L::B_KVD, par))) break;
-        tc_fence_after();
-        issue_sdp(n + 1, 0);
-        commit(L::B_SD0);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint32_t oa = ((k / 4) * L::HALF + (k % 4) * 32) >> 4;
+        const uint32_t ob = (k * 16 * 128) >> 4;
+        if (elect_one()) mma_ss(tDK, dS_k + oa, dQ_mn + so + ob, L::IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
       }
+      commit(L::B_QDE + stg);                   // dK is the last reader of Q_i, dO_i
     }
     if (total > 0) {
       commit(L::B_DONE);                        // also drains every issued product
@@ -557,6 +544,35 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         mbar_wait(bar(L::B_QD + (n & 1)), uint32_t((n >> 1) & 1), nullptr);
     }
     __syncwarp();
+  }
+
+  if (warp == 10) {
+    // ======================= lse / delta stager ==============================
+    // lane l stages query rows l, l + 32, l + 64, l + 96 of each block once
+    // every elementwise thread arrived on B_PB of the block before (its last
+    // read of those values); the loads go out before that wait
+    float* lse2_s = reinterpret_cast<float*>(smem + L::OFF_LD);
+    float* delta_s = lse2_s + 128;
+    for (int n = 0; n < total; ++n) {
+      const int hq = hkv * G + n / nblk, qb = (i_lo + n % nblk) * 128;
+      float l2[4], dl[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int q = qb + lane + 32 * u;
+        const bool qv = q < p.Nq;
+        const float l = qv ? __ldg(p.lse + (size_t(b) * p.Hq + hq) * p.Nq + q) : 0.f;
+        l2[u] = (qv && l > -CUDART_INF_F) ? l * 1.4426950408889634f : 0.f;
+        dl[u] = qv ? __ldg(p.delta + (size_t(b) * p.Hq + hq) * p.Nq + q) : 0.f;
+      }
+      if (n > 0 && !__all_sync(0xffffffffu, mbar_wait(bar(L::B_PB), uint32_t((n - 1) & 1), abort_flag)))
+        break;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        lse2_s[lane + 32 * u] = l2[u];
+        delta_s[lane + 32 * u] = dl[u];
+      }
+      mbar_arrive(bar(L::B_LD));
+    }
   }
 
   tc_fence_before();
