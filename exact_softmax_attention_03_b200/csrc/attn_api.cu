@@ -579,7 +579,9 @@ int attn_merge(const float* o_parts, const float* lse_parts, int R, void* o, flo
   int dev = 0;
   int rc = check_device(&dev);
   if (rc != ATTN_OK) return rc;
-  const unsigned grid = unsigned((rows * 32 + 255) / 256);
+  // one warp per (b, head, 32 query rows)
+  const long long warps = static_cast<long long>(B) * Hq * ((Nq + 31) / 32);
+  const unsigned grid = unsigned((warps * 32 + 255) / 256);
   uint16_t* ob = static_cast<uint16_t*>(o);
   // part count rounded up to a compile-time bound: all loads go out at once
   auto go = [&](auto dtag, auto rtag) {
