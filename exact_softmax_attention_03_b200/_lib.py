@@ -6,7 +6,13 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libattn.so")
+# ATTN_LIBRARY=debug selects the bounds-checking debug build (libattn_debug.so,
+# see attn_debug_checks in include/attn.h); the default is the release build.
+LIB_NAMES = {"release": "libattn.so", "debug": "libattn_debug.so"}
+VARIANT = os.environ.get("ATTN_LIBRARY", "release")
+if VARIANT not in LIB_NAMES:
+    raise RuntimeError(f"ATTN_LIBRARY={VARIANT!r}: expected one of {sorted(LIB_NAMES)}")
+LIB_PATH = os.path.join(_HERE, LIB_NAMES[VARIANT])
 
 ATTN_OK = 0
 ATTN_ERR_INVALID_ARG = 1
@@ -14,6 +20,7 @@ ATTN_ERR_UNSUPPORTED = 2
 ATTN_ERR_CUDA = 3
 ATTN_ERR_TIMEOUT = 4
 ATTN_ERR_WORKSPACE = 5
+ATTN_ERR_INTERNAL = 6
 
 # Size of the fixed device scratch behind attn_decode_noalloc (include/attn.h).
 ATTN_DECODE_NOALLOC_SCRATCH_BYTES = 8 << 20
@@ -25,6 +32,7 @@ STATUS_NAMES = {
     ATTN_ERR_CUDA: "ATTN_ERR_CUDA",
     ATTN_ERR_TIMEOUT: "ATTN_ERR_TIMEOUT",
     ATTN_ERR_WORKSPACE: "ATTN_ERR_WORKSPACE",
+    ATTN_ERR_INTERNAL: "ATTN_ERR_INTERNAL",
 }
 
 _vp = ctypes.c_void_p
@@ -52,6 +60,7 @@ SIGNATURES = {
     "attn_device_status": (_i, [_vp]),
     "attn_selftest_wait_timeout": (_i, [_vp]),
     "attn_launch_count": (ctypes.c_ulonglong, []),
+    "attn_debug_checks": (_i, []),
 }
 
 _lib = None

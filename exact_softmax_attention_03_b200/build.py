@@ -1,6 +1,7 @@
 """Compile the CUDA library ``libattn.so`` in-tree for sm_100a.
 
-Usage: ``python -m exact_softmax_attention_03_b200.build [--verbose]``.
+Usage: ``python -m exact_softmax_attention_03_b200.build [--verbose] [--debug]``
+(``--debug``: the bounds-checking debug build, ``libattn_debug.so``).
 The shared object is written next to this file, so it travels with the
 source tree; nothing is installed elsewhere.
 """
@@ -20,6 +21,10 @@ DEPS = [os.path.join(HERE, "csrc", f) for f in
          "backward_kernels.cuh", "merge_kernel.cuh")] + \
        [os.path.join(ROOT, "include", "attn.h")]
 LIB = os.path.join(HERE, "libattn.so")
+# the bounds-checking debug build (never the default): every kernel checks its
+# computed global indices and its roles' stage counts (include/attn.h,
+# attn_debug_checks)
+LIB_DEBUG = os.path.join(HERE, "libattn_debug.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -36,17 +41,24 @@ def nvcc_path() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(f) <= t for f in DEPS if os.path.exists(f))
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
-    cmd = [nvcc_path(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-o", LIB + ".tmp", SRC]
+def build(force: bool = False, verbose: bool = False, debug: bool | None = None) -> str:
+    """Compile the release library, or the bounds-checking debug build with
+    ``debug=True`` (default: the variant ATTN_LIBRARY selects)."""
+    if debug is None:
+        debug = os.environ.get("ATTN_LIBRARY", "release") == "debug"
+    lib = LIB_DEBUG if debug else LIB
+    if not force and up_to_date(lib):
+        return lib
+    cmd = [nvcc_path(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-o", lib + ".tmp", SRC]
+    if debug:
+        cmd += ["-DATTN_DEBUG_BOUNDS=1"]
     if verbose:
         cmd += ["-Xptxas", "-v"]
     res = subprocess.run(cmd, capture_output=True, text=True)
@@ -54,10 +66,9 @@ def build(force: bool = False, verbose: bool = False) -> str:
         raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + res.stdout + res.stderr)
     if verbose:
         sys.stderr.write(res.stdout + res.stderr)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(lib + ".tmp", lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force=True, verbose="--verbose" in sys.argv)
-    print(LIB)
+    print(build(force=True, verbose="--verbose" in sys.argv, debug="--debug" in sys.argv))

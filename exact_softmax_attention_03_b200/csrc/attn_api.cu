@@ -110,6 +110,23 @@ int make_map(CUtensorMap* map, const void* base, int d, int H, int N, int B, int
   return ATTN_OK;
 }
 
+// Page pool [num_pages, page_size, H, d] as a 5-D tensor {64, d/64, H, page_size,
+// num_pages}: one box of {64, d/64, 1, box_rows, 1} brings box_rows rows of one
+// page, every 64-column block of each row.
+int make_map_pool(CUtensorMap* map, const void* base, int d, int H, int ps, int np, int box_rows) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[5] = {64, cuuint64_t(d / 64), cuuint64_t(H), cuuint64_t(ps), cuuint64_t(np)};
+  cuuint64_t strides[4] = {128, cuuint64_t(d) * 2, cuuint64_t(H) * d * 2, cuuint64_t(ps) * H * d * 2};
+  cuuint32_t box[5] = {64, cuuint32_t(d / 64), 1, cuuint32_t(box_rows), 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return ATTN_OK;
+}
+
 bool finite_pos(float x) { return std::isfinite(x) && x > 0.f; }
 
 constexpr long long kMaxIndex = (1ll << 31) - 1;
@@ -195,6 +212,9 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
       p.vl_hg = hg;
       if (kv_heads * kv_per_seq_head <= 96.0 * (1 << 20)) break;
     }
+#ifdef ATTN_VL_HG
+    if (p.nbh_seq % ATTN_VL_HG == 0) p.vl_hg = ATTN_VL_HG;
+#endif
   }
   const long long items = static_cast<long long>(p.n_units) * p.n_bh;
   if (items > kMaxIndex) return fail(ATTN_ERR_INVALID_ARG, "problem too large for one launch");
@@ -311,8 +331,8 @@ int launch_decode_kernels(attn::DecodeParams& p, const void* k_cache, const void
   int rc;
   if constexpr (PAGED) {
     const int rows = p.page_size < 128 ? p.page_size : 128;
-    if ((rc = make_map(&mk, k_cache, D, p.Hkv, p.page_size, p.num_pages, rows)) != ATTN_OK) return rc;
-    if ((rc = make_map(&mv, v_cache, D, p.Hkv, p.page_size, p.num_pages, rows)) != ATTN_OK) return rc;
+    if ((rc = make_map_pool(&mk, k_cache, D, p.Hkv, p.page_size, p.num_pages, rows)) != ATTN_OK) return rc;
+    if ((rc = make_map_pool(&mv, v_cache, D, p.Hkv, p.page_size, p.num_pages, rows)) != ATTN_OK) return rc;
   } else {
     if ((rc = make_map(&mk, k_cache, D, p.Hkv, p.Lmax, p.B)) != ATTN_OK) return rc;
     if ((rc = make_map(&mv, v_cache, D, p.Hkv, p.Lmax, p.B)) != ATTN_OK) return rc;
@@ -735,9 +755,14 @@ int attn_device_status(cudaStream_t stream) {
   if (val == attn::kStatusBadInput)
     return fail(ATTN_ERR_INVALID_ARG, "a device-side check failed (inconsistent cu_seqlens): "
                                       "the offending sequences were skipped");
+  if (val == attn::kStatusBounds)
+    return fail(ATTN_ERR_INTERNAL, "a bounds or protocol check of the debug build failed: "
+                                   "the access was skipped");
   if (val != 0) return fail(ATTN_ERR_TIMEOUT, "a device-side wait timed out");
   return ok();
 }
+
+int attn_debug_checks(void) { return attn::kDebugBounds ? 1 : 0; }
 
 int attn_selftest_wait_timeout(cudaStream_t stream) {
   int dev = 0;

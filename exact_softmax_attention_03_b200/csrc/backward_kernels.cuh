@@ -140,14 +140,17 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p) {
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (in_bounds(static_cast<long long>(base) + EPL - 1, rows * D)) {
 #pragma unroll
-  for (int e = 0; e < EPL; ++e) p.dq_acc[base + e] = 0.f;   // slice `row` of the buffer
+    for (int e = 0; e < EPL; ++e) p.dq_acc[base + e] = 0.f;   // slice `row` of the buffer
+  }
   if (lane == 0) {
     const int h = int(row % p.Hq);
     const long long bq = row / p.Hq;                         // b * Nq + q
     const int q = int(bq % p.Nq);
     const int b = int(bq / p.Nq);
-    p.delta[(size_t(b) * p.Hq + h) * p.Nq + q] = acc;
+    const size_t di = (size_t(b) * p.Hq + h) * p.Nq + q;
+    if (in_bounds(static_cast<long long>(di), rows)) p.delta[di] = acc;
   }
 }
 
@@ -177,6 +180,8 @@ __global__ void __launch_bounds__(256) bwd_finalize_kernel(const BwdParams p) {
     const int ql = idx / (D / 8), g = idx % (D / 8);
     const int q = q0 + ql;
     if (q >= p.Nq) continue;
+    if (!in_bounds((static_cast<long long>(b) * p.Nq + q) * p.Hq + hq, static_cast<long long>(p.B) * p.Nq * p.Hq))
+      continue;
     const float4 a = tile[2 * g][ql], c = tile[2 * g + 1][ql];
     uint4 v;
     v.x = pack_bf16x2(a.x, a.y);
@@ -211,8 +216,11 @@ struct BwdLayout {
   static constexpr int B_DONE = 12;  // every dK / dV product complete
   static constexpr int B_LD = 13;    // block lse2 / delta values in shared memory (32 arrivals)
   static constexpr int NBAR = 14;
-  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;      // [0] TMEM base, [1] abort flag
-  static constexpr int BYTES = OFF_MISC + 16;
+  // [0] TMEM base, [1] abort flag; [2..4] query blocks the producer loaded, the
+  // elementwise warps and the issuer completed (compared at the end of the CTA
+  // in the bounds-checking debug build)
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int BYTES = OFF_MISC + 32;
   static constexpr int SMEM_ALLOC = BYTES + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_ST = 0, COL_DPT = 128, COL_DV = 256, COL_DK = 256 + D;
@@ -362,6 +370,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       tc_fence_before();
       mbar_arrive(bar(L::B_PB));
+      if (t == 0) reinterpret_cast<volatile int*>(smem + L::OFF_MISC)[3] = n + 1;
     }
     // ---- dK, dV of this key row ---------------------------------------------
     const bool have = ok && total > 0 &&
@@ -386,7 +395,10 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
             for (int e = 0; e < 32; ++e) r[e] = 0u;
           }
-          if (key >= p.Nk) continue;
+          if (key >= p.Nk ||
+              !in_bounds((static_cast<long long>(b) * p.Nk + key) * p.Hkv + hkv,
+                         static_cast<long long>(p.B) * p.Nk * p.Hkv))
+            continue;
 #pragma unroll
           for (int e = 0; e < 4; ++e)
             dst[4 * c + e] = make_uint4(
@@ -412,7 +424,8 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(bar(L::B_QF));
-      if (q < p.Nq) {
+      if (q < p.Nq && in_bounds((static_cast<long long>(b) * p.Hq + hq) * p.Nq + q,
+                                static_cast<long long>(p.B) * p.Hq * p.Nq)) {
         // chunk e of query q: the warp's 32 queries are 32 adjacent float4
         float4* dst = reinterpret_cast<float4*>(p.dq_acc) + (size_t(b) * p.Hq + hq) * (D / 4) * p.Nq + q;
 #pragma unroll
@@ -504,6 +517,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (elect_one()) mma_ss(tDK, dS_k + oa, dQ_mn + so + ob, L::IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
       }
       commit(L::B_QDE + stg);                   // dK is the last reader of Q_i, dO_i
+      if (lane == 0) reinterpret_cast<volatile int*>(smem + L::OFF_MISC)[4] = n + 1;
     }
     if (total > 0) {
       commit(L::B_DONE);                        // also drains every issued product
@@ -538,6 +552,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         }
         issued = n + 1;
       }
+      reinterpret_cast<volatile int*>(smem + L::OFF_MISC)[2] = issued;
       // no copy may still be landing at exit
       mbar_wait(bar(L::B_KV), 0, nullptr);
       for (int n = max(0, issued - 2); n < issued; ++n)
@@ -577,6 +592,11 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
   tc_fence_before();
   __syncthreads();
+  if (kDebugBounds && threadIdx.x == 0 && *abort_flag == 0 && total > 0) {
+    // every role went through all the CTA's query blocks
+    const volatile int* cnt = reinterpret_cast<const volatile int*>(smem + L::OFF_MISC);
+    (void)(same_count(cnt[2], total) && same_count(cnt[3], total) && same_count(cnt[4], total));
+  }
   if (warp == 8) {
     tc_fence_after();
     tmem_dealloc(tmem, L::TMEM_COLS);

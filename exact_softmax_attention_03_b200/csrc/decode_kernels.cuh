@@ -22,6 +22,17 @@
 
 namespace attn {
 
+// 5-D tiled TMA load (paged pool viewed as {64, d/64, Hkv, page rows, pages}).
+__device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1, int c2, int c3, int c4) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
+        "r"(c4), "r"(bar)
+      : "memory");
+}
+
 struct DecodeParams {
   const uint16_t* q;        // [B, Hq, D] bf16
   const uint16_t* k;        // [B, Lmax, Hkv, D] bf16 (paged: [num_pages, page_size, Hkv, D])
@@ -80,6 +91,8 @@ struct DecLayout {
   // barriers: full[STAGES], empty[STAGES], consumer sync, drain
   static constexpr int NBAR = 2 * STAGES + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;                 // abort flag
+  // [1] stages the producer loaded, [2] stages the consumers used (compared at
+  // the end of the CTA in the bounds-checking debug build)
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = BYTES + 1024;
 };
@@ -181,7 +194,9 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     int page_next = 0;
     auto fetch_page = [&](const DecItem& w, int s) -> int {
       const int t = w.k_first + 128 * s + lane * rows;
-      return t < w.hi ? __ldg(p.block_table + size_t(w.b) * p.pages_per_seq + t / ps) : p.num_pages;
+      const long long ti = static_cast<long long>(w.b) * p.pages_per_seq + t / ps;
+      return t < w.hi && in_bounds(ti, static_cast<long long>(p.B) * p.pages_per_seq)
+                 ? __ldg(p.block_table + ti) : p.num_pages;
     };
     for (int item = blockIdx.x; alive && item < n_items; item += gridDim.x) {
       DecItem w;
@@ -206,13 +221,13 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             }
           }
         } else if (box_lane) {
+          // one copy per page brings every 64-column block of its rows: the
+          // stage image is [row][block][64] (128-byte line = row * D/64 + block)
           const int r0 = lane * rows;
           const int prow = (key0 + r0) % ps;
-          for (int c = 0; c < D / 64; ++c) {
-            const uint32_t off = slot * L::TILE + c * L::HALF + r0 * 128;
-            tma_load_4d(sb + L::OFF_K + off, &tmK, bar(B_FULL + slot), c * 64, w.hkv, prow, page_cur);
-            tma_load_4d(sb + L::OFF_V + off, &tmV, bar(B_FULL + slot), c * 64, w.hkv, prow, page_cur);
-          }
+          const uint32_t off = slot * L::TILE + r0 * (D / 64) * 128;
+          tma_load_5d(sb + L::OFF_K + off, &tmK, bar(B_FULL + slot), 0, 0, w.hkv, prow, page_cur);
+          tma_load_5d(sb + L::OFF_V + off, &tmV, bar(B_FULL + slot), 0, 0, w.hkv, prow, page_cur);
         }
         __syncwarp();
       }
@@ -220,6 +235,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     // no copy may still be landing at exit: wait for the last phase of each stage
     for (int i = max(0, st - L::STAGES); i < st; ++i)
       mbar_wait(bar(B_FULL + i % L::STAGES), uint32_t(i / L::STAGES) & 1u, nullptr);
+    if (lane == 0) reinterpret_cast<volatile int*>(smem + L::OFF_MISC)[1] = st;
     __syncwarp();
   } else {
     // ======================= consumer warps ==================================
@@ -243,6 +259,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       // query rows of this group tile -> shared memory (bf16, 16 bytes per thread)
       for (int i = threadIdx.x; i < GT * D / 8; i += 256) {
         const int g = i / (D / 8), c = i % (D / 8);
+        if (!in_bounds((static_cast<long long>(w.b) * p.Hq + w.hq0 + g), static_cast<long long>(p.B) * p.Hq))
+          continue;
         *reinterpret_cast<uint4*>(smem + L::OFF_Q + (g * D + 8 * c) * 2) =
             *reinterpret_cast<const uint4*>(p.q + (size_t(w.b) * p.Hq + w.hq0 + g) * D + 8 * c);
       }
@@ -274,7 +292,13 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           // touches 8 different 16-byte bank groups
           const int ci = dh ? ((i + NCH / 2) % NCH) : i;
           const int c = dh * NCH + ci;                     // chunk of the full row
-          const uint32_t kaddr = ks + (c / 8) * L::HALF + row * 128 + (((c % 8) ^ (row & 7)) * 16);
+          uint32_t kaddr;
+          if constexpr (PAGED) {
+            const int line = row * (D / 64) + c / 8;
+            kaddr = ks + line * 128 + (((c % 8) ^ (line & 7)) * 16);
+          } else {
+            kaddr = ks + (c / 8) * L::HALF + row * 128 + (((c % 8) ^ (row & 7)) * 16);
+          }
           const uint4 kv = lds128(kaddr);
 #pragma unroll
           for (int g = 0; g < GT; ++g) {
@@ -325,7 +349,13 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
 #pragma unroll 4
         for (int kk = 0; kk < 16; ++kk) {
           const int r = 16 * warp + kk;
-          const uint32_t va = vbase + r * 128 + (((vc % 8) ^ (r & 7)) * 16);
+          uint32_t va;
+          if constexpr (PAGED) {
+            const int line = r * (D / 64) + vc / 8;
+            va = vs + line * 128 + (((vc % 8) ^ (line & 7)) * 16) + ((d0 * 2) % 16);
+          } else {
+            va = vbase + r * 128 + (((vc % 8) ^ (r & 7)) * 16);
+          }
           uint32_t v2[EPL / 2];
           if constexpr (EPL == 4) {
             asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v2[0]), "=r"(v2[1]) : "r"(va));
@@ -373,6 +403,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           }
         }
         const size_t prow = (size_t(w.b) * p.Hq + w.hq0 + g) * p.S + w.split;
+        const long long n_part = static_cast<long long>(p.B) * p.Hq * p.S;   // partial rows
+        if (!in_bounds(static_cast<long long>(prow), n_part)) continue;
         p.ws_acc[prow * D + dd] = a;
         if (dd == 0) {
           p.ws_ml[prow * 2 + 0] = M;
@@ -381,8 +413,13 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       }
       if (!(ok = consumer_sync())) break;
     }
+    if (threadIdx.x == 0) reinterpret_cast<volatile int*>(smem + L::OFF_MISC)[2] = st;
   }
   __syncthreads();
+  if (kDebugBounds && threadIdx.x == 0 && *abort_flag == 0) {
+    const volatile int* cnt = reinterpret_cast<const volatile int*>(smem + L::OFF_MISC);
+    (void)same_count(cnt[1], cnt[2]);                  // stages loaded = stages used
+  }
 }
 
 // Combine kernel: one warp per (b, hq). grid = ceil(B * Hq / 4), block = 128.
@@ -393,6 +430,7 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
   const int lane = threadIdx.x & 31;
   const int bh = blockIdx.x * 4 + warp;
   if (bh >= p.B * p.Hq) return;
+  if (!in_bounds(bh, static_cast<long long>(p.B) * p.Hq)) return;
   const int S = p.S;
   const float* ml = p.ws_ml + size_t(bh) * S * 2;
 

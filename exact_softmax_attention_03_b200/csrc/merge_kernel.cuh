@@ -70,7 +70,8 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const float* __restrict
   const float inv = L > 0.f ? 1.f / L : 0.f;
 #pragma unroll
   for (int r = 0; r < RMAX; ++r) w[r] *= inv;
-  if (lse != nullptr && lane < nrows) lse[lrow] = L > 0.f ? M + logf(L) : -CUDART_INF_F;
+  if (lse != nullptr && lane < nrows && in_bounds(static_cast<long long>(lrow), static_cast<long long>(rows)))
+    lse[lrow] = L > 0.f ? M + logf(L) : -CUDART_INF_F;
 
   // 2. the rows, U at a time
   const size_t row0 = (size_t(b) * Nq + q0) * H + h;         // row (b, q0, h) of [B, Nq, H]
@@ -115,6 +116,9 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const float* __restrict
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       if (i + u >= nrows) break;
+      if (!in_bounds(static_cast<long long>(row0) + static_cast<long long>(i + u) * H,
+                     static_cast<long long>(rows)))
+        continue;
       uint16_t* d = dst + (i + u) * rstride;
       if constexpr (EPL == 4) {
         *reinterpret_cast<uint2*>(d) = make_uint2(pack_bf16x2(acc[u][0], acc[u][1]),

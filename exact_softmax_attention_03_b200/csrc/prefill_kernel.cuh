@@ -76,11 +76,15 @@ struct FwdLayout {
   static constexpr int B_DRAIN = B_OE + 2;
   static constexpr int NBAR = B_DRAIN + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // [0] TMEM base, [1] abort flag, [2] items
+  // per-role stage counts compared at the end of the CTA (debug build):
+  // [0] K/V stages loaded, [1] K/V stages consumed by the issuer, [2..3] P.V
+  // products per tile, [4..5] score tiles the softmax warps processed per tile
+  static constexpr int OFF_DBG = OFF_MISC + 16;
   // packed-sequence schedule: sequences sorted by row units (longest first),
   // per-unit-level sequence counts, and the first item of each level
   static constexpr int VL_MAX_SEQS = kVlMaxSeqs;
   static constexpr int VL_MAX_UNITS = kVlMaxUnits;
-  static constexpr int OFF_VL = OFF_MISC + 16;                           // VarlenTables
+  static constexpr int OFF_VL = OFF_DBG + 32;                            // VarlenTables
   static constexpr int BYTES = OFF_VL + 4 * kVlInts;
   static constexpr int SMEM_ALLOC = BYTES + 1024;       // slack for 1024-byte alignment
   static constexpr uint32_t TMEM_COLS = 512;
@@ -470,17 +474,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           for (int c = 0; c < 128; ++c)
             if (c < lo_rel || c > hi_rel) s[c] = -CUDART_INF_F;
         }
-        // row max: 8 independent chains
+        // row max: 8 independent chains of three-input maxima
         float mx[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) mx[i] = s[i];
+        for (int i = 0; i < 8; ++i) mx[i] = max3f(s[i], s[8 + i], s[16 + i]);
 #pragma unroll
-        for (int c = 8; c < 128; c += 8) {
+        for (int c = 24; c < 120; c += 16) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[c + i]);
+          for (int i = 0; i < 8; ++i) mx[i] = max3f(mx[i], s[c + i], s[c + 8 + i]);
         }
-        const float mb = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[120 + i]);
+        const float mb = max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]),
+                               fmaxf(mx[6], mx[7]));
         // Lazy rescale: keep the old maximum while the new one exceeds it by at
         // most 8 in log2 units (P values stay <= 256); the final O / l is exact
         // whichever maximum was used.
@@ -570,7 +576,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
         for (int e = 0; e < D; ++e) o[e] = 0u;
       }
-      if (r < T.nq) {
+      const long long o_rows = VARLEN ? p.total_q : static_cast<long long>(p.B) * p.Nq;
+      if (r < T.nq && in_bounds(VARLEN ? w.q0 + r : static_cast<long long>(w.b) * p.Nq + r, o_rows) &&
+          in_bounds(T.hq, p.Hq)) {
         const float inv = (l > 0.f) ? 1.f / l : 0.f;
         const size_t orow = VARLEN ? size_t(w.q0) + r : size_t(w.b) * p.Nq + r;
         const size_t obase = (orow * p.Hq + T.hq) * D;
@@ -592,11 +600,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             dst[e] = v;
           }
         }
-        if (p.lse != nullptr)
-          p.lse[VARLEN ? size_t(T.hq) * p.total_q + w.q0 + r : (size_t(w.b) * p.Hq + T.hq) * p.Nq + r] =
-              (l > 0.f) ? fmaf(m, p.scale, __log2f(l) * 0.6931471805599453f) : -CUDART_INF_F;
+        const size_t li = VARLEN ? size_t(T.hq) * p.total_q + w.q0 + r : (size_t(w.b) * p.Hq + T.hq) * p.Nq + r;
+        if (p.lse != nullptr && in_bounds(static_cast<long long>(li), static_cast<long long>(p.Hq) * o_rows))
+          p.lse[li] = (l > 0.f) ? fmaf(m, p.scale, __log2f(l) * 0.6931471805599453f) : -CUDART_INF_F;
       }
     }
+    if (row == 0) reinterpret_cast<volatile int*>(smem + L::OFF_DBG)[4 + t] = count;
   } else {
   // warps 8-11 release registers to the softmax warpgroups (the release is
   // larger than the softmax groups' increase)
@@ -687,6 +696,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       commit(L::B_DRAIN);
       mbar_wait(bar(L::B_DRAIN), 0, nullptr);
       __syncwarp();
+      if (lane == 0) {
+        volatile int* dbg = reinterpret_cast<volatile int*>(smem + L::OFF_DBG);
+        dbg[1] = kv;
+        dbg[2] = pv[0];
+        dbg[3] = pv[1];
+      }
     }
     __syncwarp();
   } else if (warp == 9) {
@@ -708,16 +723,26 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (qi > 0 && !(alive = mbar_wait(bar(L::B_QE), uint32_t((qi - 1) & 1), abort_flag))) break;
         mbar_arrive_expect_tx(bar(L::B_Q), 2 * L::TILE);
 #pragma unroll
-        for (int t = 0; t < 2; ++t)
+        for (int t = 0; t < 2; ++t) {
+          // an active tile's first row lies inside Q (an inactive one reads
+          // zeros past the end, which is what the copy engine gives there)
+          if (w.tile[t].active) {
+            (void)in_bounds(w.q0 + w.tile[t].row0, VARLEN ? p.total_q : p.Nq);
+            (void)in_bounds(w.tile[t].hq, p.Hq);
+          }
           for (int c = 0; c < D / 64; ++c)
             tma_load_4d(sb + L::OFF_Q + t * L::TILE + c * L::HALF, &tmQ, bar(L::B_Q), c * 64,
                         w.tile[t].hq, w.q0 + w.tile[t].row0, w.bc);
+        }
+        (void)in_bounds(w.bc, VARLEN ? 1 : p.B);
+        (void)in_bounds(w.hkv, p.Hkv);
         ++qi;
         for (int it = 0; it < w.U; ++it, ++kv) {
           const int j = w.ubhi - 1 - it;
           const int slot = kv % L::STAGES;
           const uint32_t ph = uint32_t(kv / L::STAGES) & 1u;
           if (!(alive = mbar_wait(bar(L::B_KE + slot), ph ^ 1u, abort_flag))) break;
+          (void)in_bounds(w.k0 + j * 128, VARLEN ? p.total_k : p.Nk);   // the tile's first key
           mbar_arrive_expect_tx(bar(L::B_KF + slot), L::TILE);
           for (int c = 0; c < D / 64; ++c)
             tma_load_4d(sb + L::OFF_K + slot * L::TILE + c * L::HALF, &tmK, bar(L::B_KF + slot),
@@ -738,6 +763,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         mbar_wait(bar(L::B_KF + it % L::STAGES), uint32_t(it / L::STAGES) & 1u, nullptr);
       for (int it = max(0, issued_v - L::STAGES); it < issued_v; ++it)
         mbar_wait(bar(L::B_VF + it % L::STAGES), uint32_t(it / L::STAGES) & 1u, nullptr);
+      reinterpret_cast<volatile int*>(smem + L::OFF_DBG)[0] = issued_v;
     }
     __syncwarp();
   }
@@ -748,6 +774,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   // the only increase, the softmax groups' at the start, is always granted)
   tc_fence_before();
   __syncthreads();
+  if (kDebugBounds && threadIdx.x == 0 && *abort_flag == 0) {
+    // every role walked the same stages: loads = issues, P.V products = score
+    // tiles the softmax warps processed, per tile
+    const volatile int* dbg = reinterpret_cast<const volatile int*>(smem + L::OFF_DBG);
+    (void)(same_count(dbg[0], dbg[1]) && same_count(dbg[2], dbg[4]) && same_count(dbg[3], dbg[5]));
+  }
   if (warp == 8) {
     tc_fence_after();
     tmem_dealloc(tmem, L::TMEM_COLS);

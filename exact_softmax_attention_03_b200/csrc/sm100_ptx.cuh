@@ -14,7 +14,32 @@ __device__ int g_attn_status;
 
 constexpr int kStatusTimeout = 4;                     // == ATTN_ERR_TIMEOUT
 constexpr int kStatusBadInput = 1;                    // == ATTN_ERR_INVALID_ARG (device-side check)
+constexpr int kStatusBounds = 6;                      // == ATTN_ERR_INTERNAL (debug-build check)
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;   // 1 s per wait
+
+// Checks of the bounds-checking debug build (compiled with ATTN_DEBUG_BOUNDS;
+// the default build compiles them away). in_bounds(i, n): whether index i lies
+// in [0, n); same_count(a, b): whether two roles' counts of one protocol agree.
+// On a violation the status word records kStatusBounds and the caller skips
+// the access it guards: nothing traps, and the host reads the code through
+// attn_device_status().
+#ifdef ATTN_DEBUG_BOUNDS
+__device__ __forceinline__ bool in_bounds(long long i, long long n) {
+  if (i >= 0 && i < n) return true;
+  atomicExch(&g_attn_status, kStatusBounds);
+  return false;
+}
+__device__ __forceinline__ bool same_count(long long a, long long b) {
+  if (a == b) return true;
+  atomicExch(&g_attn_status, kStatusBounds);
+  return false;
+}
+constexpr bool kDebugBounds = true;
+#else
+__device__ __forceinline__ constexpr bool in_bounds(long long, long long) { return true; }
+__device__ __forceinline__ constexpr bool same_count(long long, long long) { return true; }
+constexpr bool kDebugBounds = false;
+#endif
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

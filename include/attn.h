@@ -64,7 +64,10 @@ typedef enum {
   ATTN_ERR_UNSUPPORTED = 2,   /* device is not sm_100, or head dim not in {64, 128} */
   ATTN_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed (message has the code) */
   ATTN_ERR_TIMEOUT = 4,       /* a bounded device-side wait gave up (see attn_device_status) */
-  ATTN_ERR_WORKSPACE = 5      /* decode or backward workspace missing or smaller than required */
+  ATTN_ERR_WORKSPACE = 5,     /* decode or backward workspace missing or smaller than required */
+  ATTN_ERR_INTERNAL = 6       /* bounds-checking debug build only: a kernel's index left its
+                                 buffer or two of its roles disagreed on a protocol count; the
+                                 access was skipped (see attn_debug_checks) */
 } attn_status;
 
 /*
@@ -249,10 +252,25 @@ const char* attn_last_error(void);
 
 /*
  * Synchronises `stream`, then reads and clears the device status word that
- * kernels set when a bounded wait gives up. Returns ATTN_OK, ATTN_ERR_TIMEOUT
- * or ATTN_ERR_CUDA (a CUDA error surfaced by the synchronisation).
+ * kernels set on a device-side failure. Returns ATTN_OK, ATTN_ERR_TIMEOUT (a
+ * bounded wait gave up), ATTN_ERR_INVALID_ARG (a device-side input check
+ * failed: inconsistent packed-sequence offsets, whose sequences were skipped),
+ * ATTN_ERR_INTERNAL (bounds-checking debug build only) or ATTN_ERR_CUDA (a
+ * CUDA error surfaced by the synchronisation).
  */
 int attn_device_status(cudaStream_t stream);
+
+/*
+ * 1 if this library is the bounds-checking debug build, else 0. That build
+ * (libattn_debug.so, compiled with ATTN_DEBUG_BOUNDS; never the default)
+ * checks, in every kernel, each computed global-memory index against the
+ * extent of the buffer it addresses and, at the end of each CTA, that the
+ * producer, tensor-core issuer and consumer roles counted the same number of
+ * pipeline stages. A failed check skips the access, records a code that
+ * attn_device_status() returns as ATTN_ERR_INTERNAL, and never traps. It is
+ * the stand-in for a memory checker on machines where none can run.
+ */
+int attn_debug_checks(void);
 
 /*
  * Diagnostic for the failure-detection path. Launches one small kernel whose

@@ -36,8 +36,21 @@ def test_header_declares_the_expected_entry_points():
         "attn_decode_workspace_bytes", "attn_merge",
         "attn_decode",
         "attn_decode_paged", "attn_decode_noalloc", "attn_last_error", "attn_device_status",
-        "attn_launch_count",
+        "attn_launch_count", "attn_debug_checks",
         "attn_selftest_wait_timeout"])
+
+
+def test_release_build_is_not_the_debug_build(lib):
+    assert lib.attn_debug_checks() == 0
+
+
+def test_debug_build_exports_the_same_symbols_and_reports_itself():
+    path = build.build(debug=True)
+    dbg = ctypes.CDLL(path)
+    for name in header_functions():
+        assert hasattr(dbg, name), name
+    dbg.attn_debug_checks.restype = ctypes.c_int
+    assert dbg.attn_debug_checks() == 1
 
 
 def test_library_exports_every_declared_symbol(lib):
