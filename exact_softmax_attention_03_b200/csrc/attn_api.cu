@@ -164,7 +164,7 @@ template <int D, bool F32OUT, bool VARLEN>
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                int Hkv, int Nq, int Nk, float scale, int causal, int window_left,
                cudaStream_t stream, int dev, const Packed* pk = nullptr) {
-  using L = attn::FwdLayout<D>;
+  using L = attn::FwdLayout<D, VARLEN>;
   CUtensorMap mq, mk, mv;
   int rc;
   // packed input: one "batch" of total rows; the kernel adds each sequence's offset
@@ -199,6 +199,27 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   }
   p.nbh_seq = p.n_bh / B;
   p.vl_hg = p.nbh_seq;
+  p.hg = p.n_bh;
+  if (!pk) {
+    // Head groups for the equal-length work list: the largest divisor of n_bh
+    // for which two consecutive groups' K/V (the keys one item touches: all of
+    // them, or the window plus a row unit) fit in 64 MB of L2. Items run level
+    // by level within a group, so every row unit of a head meets its K/V there.
+    // Groups are used only when the whole problem's K/V would not stay in
+    // L2 next to the Q and O streams (above 96 MB).
+    const double span = window_left >= 0 ? std::min<double>(Nk, double(window_left) + 256.0) : Nk;
+    const double kv_touch = span * D * 2.0 * 2.0;                 // K and V of one kv head
+    const int run = p.pair_heads ? G / 2 : G;                     // consecutive bh sharing a kv head
+    if (std::ceil(double(p.n_bh) / run) * kv_touch > 96.0 * (1 << 20)) {
+      for (int hg = p.n_bh; hg >= 1; --hg) {
+        if (p.n_bh % hg) continue;
+        p.hg = hg;
+        const double kv_heads = std::ceil(double(hg) / run);
+        if (2.0 * kv_heads * kv_touch <= 64.0 * (1 << 20)) break;
+      }
+    }
+  }
+  p.per_group = p.n_units * p.hg;
   if (pk) {
     // Head groups for the packed work list: the largest divisor of the items per
     // (sequence, unit) for which the K/V the concurrently running items touch
@@ -212,9 +233,6 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
       p.vl_hg = hg;
       if (kv_heads * kv_per_seq_head <= 96.0 * (1 << 20)) break;
     }
-#ifdef ATTN_VL_HG
-    if (p.nbh_seq % ATTN_VL_HG == 0) p.vl_hg = ATTN_VL_HG;
-#endif
   }
   const long long items = static_cast<long long>(p.n_units) * p.n_bh;
   if (items > kMaxIndex) return fail(ATTN_ERR_INVALID_ARG, "problem too large for one launch");

@@ -51,25 +51,35 @@ constexpr int kVlLvl = kVlCnt + kVlMaxUnits + 1;
 constexpr int kVlCur = kVlLvl + kVlMaxUnits + 1;
 constexpr int kVlInts = kVlCur + kVlMaxUnits + 1;
 
-template <int D>
+#ifndef ATTN_VSTAGES
+#define ATTN_VSTAGES 2
+#endif
+
+// Shared-memory layout. The packed-sequence kernel (VARLEN) also holds its
+// schedule tables, which leave room for two V stages only at D = 128; the
+// equal-length kernel has a third V stage instead (V is read by the P.V
+// products, the last in a block's issue order, so its loads have the least
+// lead time).
+template <int D, bool VARLEN = false>
 struct FwdLayout {
   static constexpr int BM = 128;                       // query rows per tile
   static constexpr int BN = 128;                       // keys per K/V tile
   static constexpr int TILE = BM * D * 2;              // bytes of a 128 x D bf16 tile
   static constexpr int HALF = 128 * 128;               // one 128-row x 64-col swizzle block
-  static constexpr int STAGES = (D == 128) ? 2 : 4;    // K/V ring depth
+  static constexpr int STAGES = (D == 128) ? 2 : 4;    // K ring depth
+  static constexpr int VSTAGES = (D == 128 && !VARLEN) ? ATTN_VSTAGES : STAGES;   // V ring depth
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + 2 * TILE;
   static constexpr int OFF_V = OFF_K + STAGES * TILE;
-  static constexpr int OFF_BAR = OFF_V + STAGES * TILE;
+  static constexpr int OFF_BAR = OFF_V + VSTAGES * TILE;
   // barrier indices
   static constexpr int B_Q = 0;                         // Q tiles loaded
   static constexpr int B_QE = 1;                        // Q tiles free (all Q.K^T done)
   static constexpr int B_KF = 2;                        // + stage
   static constexpr int B_KE = B_KF + STAGES;
-  static constexpr int B_VF = B_KE + STAGES;
-  static constexpr int B_VE = B_VF + STAGES;
-  static constexpr int B_SF = B_VE + STAGES;            // + tile
+  static constexpr int B_VF = B_KE + STAGES;            // + V stage
+  static constexpr int B_VE = B_VF + VSTAGES;
+  static constexpr int B_SF = B_VE + VSTAGES;           // + tile
   static constexpr int B_PF = B_SF + 2;                 // P written, + 2 * tile + key half
   static constexpr int B_OD = B_PF + 4;                 // P.V done, + tile
   static constexpr int B_OE = B_OD + 2;                 // O read by the epilogue, + tile
@@ -85,7 +95,7 @@ struct FwdLayout {
   static constexpr int VL_MAX_SEQS = kVlMaxSeqs;
   static constexpr int VL_MAX_UNITS = kVlMaxUnits;
   static constexpr int OFF_VL = OFF_DBG + 32;                            // VarlenTables
-  static constexpr int BYTES = OFF_VL + 4 * kVlInts;
+  static constexpr int BYTES = OFF_VL + (VARLEN ? 4 * kVlInts : 0);
   static constexpr int SMEM_ALLOC = BYTES + 1024;       // slack for 1024-byte alignment
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
@@ -112,19 +122,23 @@ struct FwdParams {
   int n_units;             // row units per (b, head-or-pair)
   int n_bh;                // number of (b, head-or-pair) combinations
   int n_items;             // n_units * n_bh
+  int hg;                  // equal lengths: (b, head-or-pair) per head group, divides n_bh
+  int per_group;           // n_units * hg: items of one head group
 };
 
 constexpr int kFwdThreads = 384;
 // Register split: the two softmax warpgroups hold a 128-score row each and
 // take kFwdRegsSoftmax per thread; the issuer/producer warpgroup gives its
-// registers up down to kFwdRegsOther (192 / 112 is the split at which neither
-// side spills). The launch must have at least kFwdRegsLaunchMin registers per
-// thread for the split to fit; the host checks the built kernel's count.
+// registers up down to kFwdRegsOther. 192 / 120 uses the launch's 168 x 384
+// registers exactly, and neither side spills (at 192 / 112 the issuer spills
+// a few bytes once it walks the head-grouped work list). The launch must have
+// at least kFwdRegsLaunchMin registers per thread for the split to fit; the
+// host checks the built kernel's count.
 #ifndef ATTN_REGS_SM
 #define ATTN_REGS_SM 192
 #endif
 #ifndef ATTN_REGS_OT
-#define ATTN_REGS_OT 112
+#define ATTN_REGS_OT 120
 #endif
 constexpr int kFwdRegsSoftmax = ATTN_REGS_SM;
 constexpr int kFwdRegsOther = ATTN_REGS_OT;
@@ -296,8 +310,13 @@ __device__ __forceinline__ void decode_item(const FwdParams& p, int item, WorkIt
     const int s = r / p.vl_hg;
     bh = vl[s] * p.nbh_seq + g * p.vl_hg + (r - s * p.vl_hg);
   } else {
-    unit = p.n_units - 1 - item / p.n_bh;                // longest rows first
-    bh = item % p.n_bh;
+    // head groups one after another (so the K/V the running items touch stays
+    // in L2), the longest rows first within a group
+    const int g = item / p.per_group;
+    const int ig = item - g * p.per_group;
+    const int lvl = ig / p.hg;
+    unit = p.n_units - 1 - lvl;
+    bh = g * p.hg + (ig - lvl * p.hg);
   }
   if (p.pair_heads) {
     const int G = p.Hq / p.Hkv;
@@ -357,20 +376,38 @@ __device__ __forceinline__ void decode_item(const FwdParams& p, int item, WorkIt
   w.U = ubhi - ublo;
 }
 
-// k-th work item of this CTA in a boustrophedon order over the items sorted
-// longest first (close to a longest-processing-time schedule); -1 when done.
-__device__ __forceinline__ int item_of(int n_items, int k) {
+// This CTA's work items, in order. The list is a sequence of head groups of
+// per_group items, the longest rows first within a group. A group's items go
+// to the CTAs in a boustrophedon (close to a longest-processing-time
+// schedule) that starts at the CTA where the previous group's items ended, so
+// the group boundaries do not pile every group's long items onto the same
+// CTAs. With one group this is the plain boustrophedon over the whole list.
+struct ItemCursor {
+  int g = 0, k = 0;                        // group, this CTA's position within it
+};
+
+__device__ __forceinline__ int next_item(ItemCursor& cur, int per_group, int n_groups) {
   const int G = int(gridDim.x);
-  const int c = (k & 1) ? (G - 1 - int(blockIdx.x)) : int(blockIdx.x);
-  const long long i = static_cast<long long>(k) * G + c;
-  return i < n_items ? int(i) : -1;
+  while (cur.g < n_groups) {
+    const int start = int((static_cast<long long>(cur.g) * per_group) % G);
+    const int c0 = int(blockIdx.x) - start;
+    const int c = c0 < 0 ? c0 + G : c0;
+    const long long i = static_cast<long long>(cur.k) * G + ((cur.k & 1) ? G - 1 - c : c);
+    if (i < per_group) {
+      ++cur.k;
+      return int(static_cast<long long>(cur.g) * per_group + i);
+    }
+    ++cur.g;
+    cur.k = 0;
+  }
+  return -1;
 }
 
 template <int D, bool F32OUT, bool VARLEN>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
-  using L = FwdLayout<D>;
+  using L = FwdLayout<D, VARLEN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -389,6 +426,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     for (int s = 0; s < L::STAGES; ++s) {
       mbar_init(bar(L::B_KF + s), 1);
       mbar_init(bar(L::B_KE + s), 1);
+    }
+    for (int s = 0; s < L::VSTAGES; ++s) {
       mbar_init(bar(L::B_VF + s), 1);
       mbar_init(bar(L::B_VE + s), 1);
     }
@@ -413,13 +452,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const uint32_t tmem = *tmem_holder;
   // the work list: closed form, or the compact list of packed sequences
   const int* vs = nullptr;
-  int n_items = p.n_items;
+  int per_group = p.per_group, n_groups = p.n_bh / p.hg;
   if constexpr (VARLEN) {
     int* vl = reinterpret_cast<int*>(smem + L::OFF_VL);
     int* vl_items = reinterpret_cast<int*>(smem + L::OFF_MISC + 8);
     build_varlen_sched(p, vl, vl_items);
     vs = vl;
-    n_items = *vl_items;
+    per_group = vl[kVlLvl + p.n_units];                 // items of one head group
+    n_groups = p.nbh_seq / p.vl_hg;
   }
 
   if (warp < 8) {
@@ -433,8 +473,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const float c2 = p.scale_log2;
     int count = 0;                          // S tiles processed so far (all items)
     bool ok = true;
-    for (int k = 0; ok; ++k) {
-      const int item = item_of(n_items, k);
+    ItemCursor cur;
+    while (ok) {
+      const int item = next_item(cur, per_group, n_groups);
       if (item < 0) break;
       WorkItem w;
       decode_item<VARLEN>(p, item, w, vs);
@@ -520,17 +561,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
               const int c = 32 * hf + i;
-              const uint64_t x = f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), C2, NMO);
-              uint64_t e;
+              float p0, p1;
               if ((i % kPolyEvery) == kPolyEvery - 1) {
-                e = exp2_poly_f2(x);
+                const uint64_t x = f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), C2, NMO);
+                const float2 ee = f2_unpack(exp2_poly_f2(x));
+                p0 = ee.x;
+                p1 = ee.y;
               } else {
-                const float2 xx = f2_unpack(x);
-                e = f2_pack(ex2_approx(xx.x), ex2_approx(xx.y));
+                const float2 xx = f2_unpack(f2_fma(f2_pack(s[2 * c], s[2 * c + 1]), C2, NMO));
+                p0 = ex2_approx(xx.x);
+                p1 = ex2_approx(xx.y);
               }
-              lacc[i & 3] = f2_add(lacc[i & 3], e);
-              const float2 ee = f2_unpack(e);
-              pk[i] = pack_bf16x2(ee.x, ee.y);
+              lacc[i & 3] = f2_add(lacc[i & 3], f2_pack(p0, p1));
+              pk[i] = pack_bf16x2(p0, p1);
             }
           }
           tmem_st32(tS + 32 * hf, pk);
@@ -551,7 +594,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           mbar_arrive(bar(L::B_PF + 2 * t + hf));
         }
         const float2 l01 = f2_unpack(f2_add(f2_add(lacc[0], lacc[1]), f2_add(lacc[2], lacc[3])));
-        l = fmaf(l, alpha, l01.x + l01.y);
+        const float lsum = l01.x + l01.y;
+        l = fmaf(l, alpha, lsum);
         ++count;
         ++n_in_item;
       }
@@ -648,8 +692,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       };
       int kv = 0, qi = 0;                   // K/V ring position, items with a Q load
       bool alive = true;
-      for (int k = 0; alive; ++k) {
-        const int item = item_of(n_items, k);
+      ItemCursor cur;
+      while (alive) {
+        const int item = next_item(cur, per_group, n_groups);
         if (item < 0) break;
         WorkItem w;
         decode_item<VARLEN>(p, item, w, vs);
@@ -657,11 +702,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (!(alive = wwait(L::B_Q, uint32_t(qi & 1)))) break;
         tc_fence_after();
         first[0] = first[1] = true;
-        int prev_j = -1, prev_slot = 0;
+        int prev_j = -1, prev_vslot = 0;
         for (int it = 0; it < w.U; ++it, ++kv) {
           const int j = w.ubhi - 1 - it;
           const int slot = kv % L::STAGES;
           const uint32_t ph = uint32_t(kv / L::STAGES) & 1u;
+          const int vslot = kv % L::VSTAGES;
+          const uint32_t vph = uint32_t(kv / L::VSTAGES) & 1u;
           if (!(alive = wwait(L::B_KF + slot, ph))) break;
           tc_fence_after();
           const uint64_t kd = dk + uint32_t(slot * (L::TILE >> 4));
@@ -670,8 +717,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             commit(L::B_SF + 0);
           }
           if (it > 0) {
-            if (tile_has(w.tile[1], prev_j) && !(alive = pv_tile(1, prev_slot))) break;
-            commit(L::B_VE + prev_slot);
+            if (tile_has(w.tile[1], prev_j) && !(alive = pv_tile(1, prev_vslot))) break;
+            commit(L::B_VE + prev_vslot);
           }
           if (tile_has(w.tile[1], j)) {
             issue_qk<D>(dS1, dq1, kd);
@@ -679,15 +726,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           }
           commit(L::B_KE + slot);
           if (it == w.U - 1) commit(L::B_QE);     // every Q.K^T of this item issued
-          if (!(alive = wwait(L::B_VF + slot, ph))) break;
+          if (!(alive = wwait(L::B_VF + vslot, vph))) break;
           tc_fence_after();
-          if (tile_has(w.tile[0], j) && !(alive = pv_tile(0, slot))) break;
+          if (tile_has(w.tile[0], j) && !(alive = pv_tile(0, vslot))) break;
           prev_j = j;
-          prev_slot = slot;
+          prev_vslot = vslot;
         }
         if (!alive) break;
-        if (tile_has(w.tile[1], prev_j) && !(alive = pv_tile(1, prev_slot))) break;
-        commit(L::B_VE + prev_slot);
+        if (tile_has(w.tile[1], prev_j) && !(alive = pv_tile(1, prev_vslot))) break;
+        commit(L::B_VE + prev_vslot);
         if (!first[0]) ++done[0];
         if (!first[1]) ++done[1];
         ++qi;
@@ -713,8 +760,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       int kv = 0, qi = 0;                   // same counters as the issuer
       int issued_k = 0, issued_v = 0;
       bool alive = true;
-      for (int k = 0; alive; ++k) {
-        const int item = item_of(n_items, k);
+      ItemCursor cur;
+      while (alive) {
+        const int item = next_item(cur, per_group, n_groups);
         if (item < 0) break;
         WorkItem w;
         decode_item<VARLEN>(p, item, w, vs);
@@ -748,10 +796,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             tma_load_4d(sb + L::OFF_K + slot * L::TILE + c * L::HALF, &tmK, bar(L::B_KF + slot),
                         c * 64, w.hkv, w.k0 + j * 128, w.bc);
           issued_k = kv + 1;
-          if (!(alive = mbar_wait(bar(L::B_VE + slot), ph ^ 1u, abort_flag))) break;
-          mbar_arrive_expect_tx(bar(L::B_VF + slot), L::TILE);
+          const int vslot = kv % L::VSTAGES;
+          const uint32_t vph = uint32_t(kv / L::VSTAGES) & 1u;
+          if (!(alive = mbar_wait(bar(L::B_VE + vslot), vph ^ 1u, abort_flag))) break;
+          mbar_arrive_expect_tx(bar(L::B_VF + vslot), L::TILE);
           for (int c = 0; c < D / 64; ++c)
-            tma_load_4d(sb + L::OFF_V + slot * L::TILE + c * L::HALF, &tmV, bar(L::B_VF + slot),
+            tma_load_4d(sb + L::OFF_V + vslot * L::TILE + c * L::HALF, &tmV, bar(L::B_VF + vslot),
                         c * 64, w.hkv, w.k0 + j * 128, w.bc);
           issued_v = kv + 1;
         }
@@ -761,8 +811,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       if (qi > 0) mbar_wait(bar(L::B_Q), uint32_t((qi - 1) & 1), nullptr);
       for (int it = max(0, issued_k - L::STAGES); it < issued_k; ++it)
         mbar_wait(bar(L::B_KF + it % L::STAGES), uint32_t(it / L::STAGES) & 1u, nullptr);
-      for (int it = max(0, issued_v - L::STAGES); it < issued_v; ++it)
-        mbar_wait(bar(L::B_VF + it % L::STAGES), uint32_t(it / L::STAGES) & 1u, nullptr);
+      for (int it = max(0, issued_v - L::VSTAGES); it < issued_v; ++it)
+        mbar_wait(bar(L::B_VF + it % L::VSTAGES), uint32_t(it / L::VSTAGES) & 1u, nullptr);
       reinterpret_cast<volatile int*>(smem + L::OFF_DBG)[0] = issued_v;
     }
     __syncwarp();

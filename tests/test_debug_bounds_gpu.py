@@ -9,8 +9,10 @@ memory checker, which cannot run on these machines.
 Here the small forward (plain, windowed, GQA, packed), decode (contiguous and
 paged), backward and merge parity tests run in a child process against the
 debug build (ATTN_LIBRARY=debug): every call must pass parity with the fp64
-oracle and leave the status word clear. Only valid inputs are used: a check
-that fails on a valid input is a bug in the kernel or in the check.
+oracle and leave the status word clear. So does the full-size MHA causal
+N = 8192 forward, the one workload here whose work list runs in head groups.
+Only valid inputs are used: a check that fails on a valid input is a bug in
+the kernel or in the check.
 """
 
 import os
@@ -62,3 +64,12 @@ def test_small_parity_cases_pass_under_the_debug_build(debug_lib):
     res = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=1800)
     assert res.returncode == 0, (res.stdout[-4000:], res.stderr[-2000:])
     assert " passed" in res.stdout
+
+
+def test_full_size_head_grouped_forward_under_the_debug_build(debug_lib):
+    env = dict(os.environ, ATTN_LIBRARY="debug")
+    cmd = [sys.executable, "-m", "pytest", "-q", "-x", "-m", "gpu", "-k", "N8192",
+           "-p", "no:cacheprovider", "tests/test_fwd_gpu.py::test_full_size_whole_head_and_late_rows"]
+    res = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=1800)
+    assert res.returncode == 0, (res.stdout[-4000:], res.stderr[-2000:])
+    assert "1 passed" in res.stdout
