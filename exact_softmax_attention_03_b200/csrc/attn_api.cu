@@ -172,6 +172,8 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   if ((rc = make_map(&mq, q, D, Hq, rq, nb)) != ATTN_OK) return rc;
   if ((rc = make_map(&mk, k, D, Hkv, rk, nb)) != ATTN_OK) return rc;
   if ((rc = make_map(&mv, v, D, Hkv, rk, nb)) != ATTN_OK) return rc;
+  CUtensorMap mo = mq;                 // O map: used by the equal-length bf16 kernel only
+  if (!VARLEN && !F32OUT && (rc = make_map(&mo, o, D, Hq, Nq, B, 32)) != ATTN_OK) return rc;
 
   attn::FwdParams p{};
   p.o = o;
@@ -220,6 +222,14 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     }
   }
   p.per_group = p.n_units * p.hg;
+  // O through staged bulk stores when a tile's walk is short (the per-item
+  // epilogue is then a large share of the time); for long walks the row
+  // stores, which take no shared-memory bandwidth from the products
+  if (!pk && !F32OUT) {
+    const double rows_keys = window_left >= 0 ? std::min<double>(Nk, window_left + 1.0)
+                             : causal ? std::max(0.0, Nk - Nq + Nq / 2.0) : double(Nk);
+    p.bulk_o = rows_keys / 128.0 + 1.0 <= ATTN_BULK_O_MAX_BLOCKS ? 1 : 0;
+  }
   if (pk) {
     // Head groups for the packed work list: the largest divisor of the items per
     // (sequence, unit) for which the K/V the concurrently running items touch
@@ -259,7 +269,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     attr_set.fetch_or(bit);
   }
-  attn::attn_fwd_kernel<D, F32OUT, VARLEN><<<unsigned(grid), attn::kFwdThreads, L::SMEM_ALLOC, stream>>>(mq, mk, mv, p);
+  attn::attn_fwd_kernel<D, F32OUT, VARLEN><<<unsigned(grid), attn::kFwdThreads, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mo, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "attn_fwd launch: %s", cudaGetErrorString(e));
   g_launches.fetch_add(1);
@@ -433,12 +443,15 @@ int launch_bwd(const void* q, const void* k, const void* v, attn::BwdParams& p, 
   const long long nbh = static_cast<long long>(p.B) * p.Hkv;
   const long long nctas = static_cast<long long>((p.Nk + 127) / 128) * nbh;
   if (nctas > kMaxIndex) return fail(ATTN_ERR_INVALID_ARG, "problem too large for one launch");
-  CUtensorMap mq, mk, mv, mdo;
+  CUtensorMap mq, mk, mv, mdo, mdk, mdv;
   int rc;
   if ((rc = make_map(&mq, q, D, p.Hq, p.Nq, p.B)) != ATTN_OK) return rc;
   if ((rc = make_map(&mk, k, D, p.Hkv, p.Nk, p.B)) != ATTN_OK) return rc;
   if ((rc = make_map(&mv, v, D, p.Hkv, p.Nk, p.B)) != ATTN_OK) return rc;
   if ((rc = make_map(&mdo, p.dout, D, p.Hq, p.Nq, p.B)) != ATTN_OK) return rc;
+  // dK, dV leave through 32-row bulk tensor stores
+  if ((rc = make_map(&mdk, p.dk, D, p.Hkv, p.Nk, p.B, 32)) != ATTN_OK) return rc;
+  if ((rc = make_map(&mdv, p.dv, D, p.Hkv, p.Nk, p.B, 32)) != ATTN_OK) return rc;
   static std::atomic<unsigned long long> attr_set{0};   // per-device bit
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(attr_set.load() & bit)) {
@@ -453,7 +466,7 @@ int launch_bwd(const void* q, const void* k, const void* v, attn::BwdParams& p, 
   // (fp32) rows take about 48 MB of L2
   const long long unit = static_cast<long long>(p.Hq / p.Hkv) * p.Nq * D * 8;
   p.bh_chunk = static_cast<int>(std::max(1ll, std::min(nbh, (48ll << 20) / unit)));
-  attn::bwd_main_kernel<D><<<unsigned(nctas), attn::kBwdThreads, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, p);
+  attn::bwd_main_kernel<D><<<unsigned(nctas), attn::kBwdThreads, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, mdk, mdv, p);
   const long long fin = static_cast<long long>(p.B) * p.Hq * ((p.Nq + attn::kFinQ - 1) / attn::kFinQ);
   attn::bwd_finalize_kernel<D><<<unsigned(fin), 256, 0, stream>>>(p);
   return ATTN_OK;

@@ -246,6 +246,7 @@ template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
                 const BwdParams p) {
   using L = BwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -376,37 +377,47 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const bool have = ok && total > 0 &&
                       __all_sync(0xffffffffu, mbar_wait(bar(L::B_DONE), 0u, abort_flag));
     if (have) tc_fence_after();
-    // tcgen05.ld is warp-collective: every lane loads; only the stores of
-    // keys inside the sequence are guarded
-    if (have || (ok && total == 0)) {
-      const size_t base = ((size_t(b) * p.Nk + min(key, p.Nk - 1)) * p.Hkv + hkv) * D;
+    // Each warp stages its 32 key rows of dV, then dK (scaled), as 4 KB blocks
+    // of 32 rows x 64 columns in the 128-byte swizzled layout of the tensor
+    // maps, in the Q ring (free once every product has completed); lane 0
+    // stores the blocks. Rows past Nk fall outside the maps and are not written.
+    const int wk0 = kb0 + 32 * warp;
+    if ((have || (ok && total == 0)) && wk0 < p.Nk) {
+      constexpr int NH = D / 64;
+      const uint32_t stg = sb + L::OFF_Q + uint32_t(warp) * (2 * NH * 4096);
 #pragma unroll
       for (int m = 0; m < 2; ++m) {                          // 0: dV, 1: dK (scaled)
-        uint4* dst = reinterpret_cast<uint4*>((m ? p.dk : p.dv) + base);
         const float f = m ? p.scale : 1.f;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t r[32];
           if (have) {
-            __syncwarp();
             tmem_ld32(tmem + lane_off + (m ? L::COL_DK : L::COL_DV) + 32 * c, r);
             tmem_wait_ld();
           } else {
 #pragma unroll
             for (int e = 0; e < 32; ++e) r[e] = 0u;
           }
-          if (key >= p.Nk ||
-              !in_bounds((static_cast<long long>(b) * p.Nk + key) * p.Hkv + hkv,
-                         static_cast<long long>(p.B) * p.Nk * p.Hkv))
-            continue;
+          const uint32_t blk = stg + uint32_t(m * NH + c / 2) * 4096u + uint32_t(lane) * 128u;
 #pragma unroll
           for (int e = 0; e < 4; ++e)
-            dst[4 * c + e] = make_uint4(
-                pack_bf16x2(__uint_as_float(r[8 * e]) * f, __uint_as_float(r[8 * e + 1]) * f),
-                pack_bf16x2(__uint_as_float(r[8 * e + 2]) * f, __uint_as_float(r[8 * e + 3]) * f),
-                pack_bf16x2(__uint_as_float(r[8 * e + 4]) * f, __uint_as_float(r[8 * e + 5]) * f),
-                pack_bf16x2(__uint_as_float(r[8 * e + 6]) * f, __uint_as_float(r[8 * e + 7]) * f));
+            st_shared_v4(blk + uint32_t(((4 * (c & 1) + e) ^ (lane & 7)) << 4),
+                         pack_bf16x2(__uint_as_float(r[8 * e]) * f, __uint_as_float(r[8 * e + 1]) * f),
+                         pack_bf16x2(__uint_as_float(r[8 * e + 2]) * f, __uint_as_float(r[8 * e + 3]) * f),
+                         pack_bf16x2(__uint_as_float(r[8 * e + 4]) * f, __uint_as_float(r[8 * e + 5]) * f),
+                         pack_bf16x2(__uint_as_float(r[8 * e + 6]) * f, __uint_as_float(r[8 * e + 7]) * f));
         }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && in_bounds(b, p.B) && in_bounds(hkv, p.Hkv)) {
+#pragma unroll
+        for (int m = 0; m < 2; ++m)
+#pragma unroll
+          for (int h = 0; h < NH; ++h)
+            tma_store_4d(m ? &tmDK : &tmDV, stg + uint32_t(m * NH + h) * 4096u, 64 * h, hkv, wk0, b);
+        bulk_commit_group();
+        bulk_wait_all();                    // shared memory outlives the stores
       }
     }
   } else if (warp < 8) {

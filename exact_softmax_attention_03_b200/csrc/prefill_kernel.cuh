@@ -54,6 +54,9 @@ constexpr int kVlInts = kVlCur + kVlMaxUnits + 1;
 #ifndef ATTN_VSTAGES
 #define ATTN_VSTAGES 2
 #endif
+#ifndef ATTN_BULK_O_MAX_BLOCKS
+#define ATTN_BULK_O_MAX_BLOCKS 16
+#endif
 
 // Shared-memory layout. The packed-sequence kernel (VARLEN) also holds its
 // schedule tables, which leave room for two V stages only at D = 128; the
@@ -71,7 +74,11 @@ struct FwdLayout {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + 2 * TILE;
   static constexpr int OFF_V = OFF_K + STAGES * TILE;
-  static constexpr int OFF_BAR = OFF_V + VSTAGES * TILE;
+  // equal-length kernel: a 32-row x 64-column O staging block per softmax warp
+  // for the bulk tensor stores of the epilogue (the packed kernel stores O
+  // directly)
+  static constexpr int OFF_OST = OFF_V + VSTAGES * TILE;
+  static constexpr int OFF_BAR = OFF_OST + (VARLEN ? 0 : 2 * HALF);
   // barrier indices
   static constexpr int B_Q = 0;                         // Q tiles loaded
   static constexpr int B_QE = 1;                        // Q tiles free (all Q.K^T done)
@@ -124,6 +131,7 @@ struct FwdParams {
   int n_items;             // n_units * n_bh
   int hg;                  // equal lengths: (b, head-or-pair) per head group, divides n_bh
   int per_group;           // n_units * hg: items of one head group
+  int bulk_o;              // equal-length bf16 O: 1 = staged bulk tensor stores, 0 = row stores
 };
 
 constexpr int kFwdThreads = 384;
@@ -406,8 +414,13 @@ __device__ __forceinline__ int next_item(ItemCursor& cur, int per_group, int n_g
 template <int D, bool F32OUT, bool VARLEN>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                const FwdParams p) {
   using L = FwdLayout<D, VARLEN>;
+  // bf16 O of the equal-length kernel can leave through shared memory and bulk
+  // tensor stores (tmO, when p.bulk_o); otherwise each thread stores its row
+  // from registers
+  constexpr bool kTmaO = !VARLEN && !F32OUT;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -621,9 +634,43 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         for (int e = 0; e < D; ++e) o[e] = 0u;
       }
       const long long o_rows = VARLEN ? p.total_q : static_cast<long long>(p.B) * p.Nq;
+      const float inv = (l > 0.f) ? 1.f / l : 0.f;
+      const bool bulk_o = kTmaO && p.bulk_o;
+      if (bulk_o) {
+        // Each warp writes its 32 rows to its own staging block, 64 columns at
+        // a time, in the 128-byte swizzled layout of the tensor map; lane 0
+        // then stores the block (rows past Nq fall outside the map and are not
+        // written). A block is rewritten only after its previous store has
+        // read it. Only warp-level synchronisation: no warp ever waits on
+        // another one here.
+        const int wr0 = T.row0 + 32 * (warp & 3);
+        if (wr0 < T.nq) {
+          const uint32_t stg = sb + L::OFF_OST + uint32_t(t) * L::HALF + uint32_t(warp & 3) * 4096u;
+          const uint32_t rbase = stg + uint32_t(lane) * 128u;
+#pragma unroll
+          for (int h = 0; h < D / 64; ++h) {
+            if (lane == 0) bulk_wait_read_all();
+            __syncwarp();
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const uint32_t* e = o + 64 * h + 8 * c;
+              st_shared_v4(rbase + uint32_t((c ^ (lane & 7)) << 4),
+                           pack_bf16x2(__uint_as_float(e[0]) * inv, __uint_as_float(e[1]) * inv),
+                           pack_bf16x2(__uint_as_float(e[2]) * inv, __uint_as_float(e[3]) * inv),
+                           pack_bf16x2(__uint_as_float(e[4]) * inv, __uint_as_float(e[5]) * inv),
+                           pack_bf16x2(__uint_as_float(e[6]) * inv, __uint_as_float(e[7]) * inv));
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && in_bounds(w.b, p.B) && in_bounds(T.hq, p.Hq)) {
+              tma_store_4d(&tmO, stg, 64 * h, T.hq, wr0, w.b);
+              bulk_commit_group();
+            }
+          }
+        }
+      }
       if (r < T.nq && in_bounds(VARLEN ? w.q0 + r : static_cast<long long>(w.b) * p.Nq + r, o_rows) &&
           in_bounds(T.hq, p.Hq)) {
-        const float inv = (l > 0.f) ? 1.f / l : 0.f;
         const size_t orow = VARLEN ? size_t(w.q0) + r : size_t(w.b) * p.Nq + r;
         const size_t obase = (orow * p.Hq + T.hq) * D;
         if constexpr (F32OUT) {
@@ -632,7 +679,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           for (int e = 0; e < D / 4; ++e)
             dst[e] = make_float4(__uint_as_float(o[4 * e]) * inv, __uint_as_float(o[4 * e + 1]) * inv,
                                  __uint_as_float(o[4 * e + 2]) * inv, __uint_as_float(o[4 * e + 3]) * inv);
-        } else {
+        } else if (!bulk_o) {
           uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) + obase);
 #pragma unroll
           for (int e = 0; e < D / 8; ++e) {
@@ -649,6 +696,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           p.lse[li] = (l > 0.f) ? fmaf(m, p.scale, __log2f(l) * 0.6931471805599453f) : -CUDART_INF_F;
       }
     }
+    // the CTA's shared memory must outlive the last O stores
+    if (kTmaO && lane == 0) bulk_wait_all();
     if (row == 0) reinterpret_cast<volatile int*>(smem + L::OFF_DBG)[4 + t] = count;
   } else {
   // warps 8-11 release registers to the softmax warpgroups (the release is

@@ -168,6 +168,24 @@ def test_full_size_whole_head_and_late_rows(w):
         assert_close(o[b, rows, hq], O, lse[b, hq, rows], L, what=(w.name, b, hq))
 
 
+def test_head_grouped_gqa_causal_sampled_rows():
+    """GQA causal without a window at N = 32768 (Hq32 Hkv8): its K/V (128 MB) is
+    above L2, so the work list runs in head groups (4 of 4 head pairs each) with
+    the rotated per-group assignment. Sampled rows of 6 heads, including the
+    shortest causal rows (they run last within each group)."""
+    B, Hq, Hkv, N, d = 1, 32, 8, 32768, 128
+    q, k, v = ai.make_qkv(B, Hq, Hkv, N, N, d, seed=ai.SEED_Q + 90)
+    o, lse = run_fwd(q, k, v, True, -1)
+    G = Hq // Hkv
+    g = torch.Generator().manual_seed(5)
+    for hq in (0, 5, 10, 17, 26, 31):
+        early = torch.randint(0, 256, (6,), generator=g).tolist()
+        rows = sorted(set(early + sample_rows(N, 12, seed=hq)))
+        O, L = oracle.oracle_attention_rows(_head(q, 0, hq), _head(k, 0, hq // G),
+                                            _head(v, 0, hq // G), 0, 0, rows, causal=True)
+        assert_close(o[0, rows, hq], O, lse[0, hq, rows], L, what=("grouped GQA", hq))
+
+
 def _scaled_keys(k, factor_of_key):
     k = k.float().clone()
     for j in range(k.shape[1]):
