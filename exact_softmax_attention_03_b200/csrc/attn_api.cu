@@ -222,14 +222,9 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     }
   }
   p.per_group = p.n_units * p.hg;
-  // O through staged bulk stores when a tile's walk is short (the per-item
-  // epilogue is then a large share of the time); for long walks the row
-  // stores, which take no shared-memory bandwidth from the products
-  if (!pk && !F32OUT) {
-    const double rows_keys = window_left >= 0 ? std::min<double>(Nk, window_left + 1.0)
-                             : causal ? std::max(0.0, Nk - Nq + Nq / 2.0) : double(Nk);
-    p.bulk_o = rows_keys / 128.0 + 1.0 <= ATTN_BULK_O_MAX_BLOCKS ? 1 : 0;
-  }
+  // equal-length bf16 O: staged bulk tensor stores (the kernel keeps the
+  // per-row stores as a launch-time alternative, p.bulk_o = 0)
+  p.bulk_o = (!pk && !F32OUT) ? 1 : 0;
   if (pk) {
     // Head groups for the packed work list: the largest divisor of the items per
     // (sequence, unit) for which the K/V the concurrently running items touch

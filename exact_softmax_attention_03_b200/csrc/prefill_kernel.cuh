@@ -54,9 +54,6 @@ constexpr int kVlInts = kVlCur + kVlMaxUnits + 1;
 #ifndef ATTN_VSTAGES
 #define ATTN_VSTAGES 2
 #endif
-#ifndef ATTN_BULK_O_MAX_BLOCKS
-#define ATTN_BULK_O_MAX_BLOCKS 16
-#endif
 
 // Shared-memory layout. The packed-sequence kernel (VARLEN) also holds its
 // schedule tables, which leave room for two V stages only at D = 128; the
@@ -417,9 +414,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                 const FwdParams p) {
   using L = FwdLayout<D, VARLEN>;
-  // bf16 O of the equal-length kernel can leave through shared memory and bulk
-  // tensor stores (tmO, when p.bulk_o); otherwise each thread stores its row
-  // from registers
+  // bf16 O of the equal-length kernel leaves through shared memory and bulk
+  // tensor stores (tmO) when p.bulk_o, which the host sets for every such
+  // launch; otherwise each thread stores its row from registers. The choice
+  // stays a launch parameter: built that way, the kernel measured 1-3 points
+  // of the bf16 peak faster than with the bulk stores fixed at compile time.
   constexpr bool kTmaO = !VARLEN && !F32OUT;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
