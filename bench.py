@@ -129,7 +129,9 @@ def recorded_traffic(kernel: str, workload: str, resized: bool = False):
 # ------------------------------------------------------------------ clocks --
 
 class ClockSampler:
-    """Samples SM clock and clock-event reasons through NVML during a region."""
+    """Samples SM clock and clock-event reasons through NVML, only while a timed
+    region is open (``timed_kernel_loop`` opens one per leg): the median is the
+    clock under load, per leg and over all legs."""
 
     REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
                0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
@@ -138,7 +140,8 @@ class ClockSampler:
 
     def __init__(self, device_index: int, period_s: float = 0.01):
         self.period = period_s
-        self.samples = []
+        self.samples = []                         # (leg label, MHz)
+        self.label = None                         # open timed region, or None
         self.reasons = 0
         self.max_mhz = None
         self._stop = threading.Event()
@@ -154,14 +157,22 @@ class ClockSampler:
 
     def _run(self):
         while not self._stop.is_set():
-            try:
-                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
-                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                self.samples.append(mhz)
-                self.reasons |= int(r) & ~0x1
-            except Exception:
-                pass
+            label = self.label
+            if label is not None:
+                try:
+                    mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                    r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                    self.samples.append((label, mhz))
+                    self.reasons |= int(r) & ~0x1
+                except Exception:
+                    pass
             time.sleep(self.period)
+
+    def open(self, label):
+        self.label = label
+
+    def close(self):
+        self.label = None
 
     def start(self):
         if self.nv is not None:
@@ -176,9 +187,17 @@ class ClockSampler:
     def summary(self):
         if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+        legs = {}
+        for label, mhz in self.samples:
+            legs.setdefault(label, []).append(mhz)
+        return {"sm_mhz": statistics.median(m for _, m in self.samples), "sm_max_mhz": self.max_mhz,
                 "reasons": [n for b, n in self.REASONS.items() if self.reasons & b],
-                "samples": len(self.samples)}
+                "samples": len(self.samples),
+                "sm_mhz_per_leg": {k: statistics.median(v) for k, v in legs.items()},
+                "scope": "timed regions only"}
+
+
+SAMPLER = None          # the run's ClockSampler (timed_kernel_loop opens and closes it)
 
 
 # -------------------------------------------------------------- dist setup --
@@ -224,7 +243,7 @@ def whole_job_rate(units_per_rank: float, ms_max: float, world: int) -> float:
 
 # ------------------------------------------------------------------ timing --
 
-def timed_kernel_loop(fn, steps, warmup, world, flush=None):
+def timed_kernel_loop(fn, steps, warmup, world, flush=None, label="leg"):
     """Per-step CUDA-event times (ms) of fn() on the current stream; returns
     (times, launches of this library inside the timed region)."""
     import exact_softmax_attention_03_b200 as ea
@@ -239,6 +258,8 @@ def timed_kernel_loop(fn, steps, warmup, world, flush=None):
     barrier(world)
     torch.cuda.synchronize()
     n0 = ea.attn_launch_count()
+    if SAMPLER is not None:
+        SAMPLER.open(label)
     for s, e in ev:
         if flush is not None:
             flush()
@@ -247,6 +268,8 @@ def timed_kernel_loop(fn, steps, warmup, world, flush=None):
         fn()
         e.record(stream)
     torch.cuda.synchronize()
+    if SAMPLER is not None:
+        SAMPLER.close()
     n1 = ea.attn_launch_count()
     barrier(world)
     status = ea.attn_device_status()
@@ -428,6 +451,12 @@ def tensor_roofline(achieved, peaks, peak_src, kernel, traffic, alg_bytes=None):
     r = {"bound": "tensor", "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
          "frac": achieved / peak_t, "peak_source": f"{peak_src} bf16_tflops (burst)",
          "kernel": kernel, "traffic": traffic}
+    if "bf16_tflops_sustained" in peaks:
+        # the timed loop runs the kernel back to back, where the SM clock settles
+        # below its burst value under the power cap: the sustained GEMM figure,
+        # measured the same way, is the like-for-like denominator
+        r["peak_sustained"] = peaks["bf16_tflops_sustained"]
+        r["frac_sustained"] = achieved / peaks["bf16_tflops_sustained"]
     if alg_bytes is not None:
         r["algorithmic_bytes"] = alg_bytes
     return r
@@ -449,7 +478,7 @@ def prefill_leg(ea, key, w, args, world, rank, dev, flush, peaks, peak_src, resi
     def fwd():
         ea.attn_fwd(q, k, v, o=o, lse=lse, causal=w.causal, window_left=w.window_left)
 
-    times, launches = timed_kernel_loop(fwd, args.steps, args.warmup, world, flush)
+    times, launches = timed_kernel_loop(fwd, args.steps, args.warmup, world, flush, label=key)
     st = time_stats(times)
     ms_max = max_over_ranks(st["mean"], world)
     flops = metrics.attn_flops(w.B, w.Hq, w.Nq, w.Nk, w.d, w.causal, w.window_left)
@@ -480,7 +509,9 @@ def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     peaks, peak_src = load_peaks()
+    global SAMPLER
     sampler = ClockSampler(torch.cuda.current_device() if world == 1 else local)
+    SAMPLER = sampler
     flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
     def flush():
@@ -526,7 +557,7 @@ def run_ours(args, world, rank, local):
         ea.attn_bwd(q, k, v, o, lse, dout, causal=w.causal, window_left=w.window_left,
                     dq=dq_t, dk=dk_t, dv=dv_t, workspace=bws)
 
-    btimes, blaunches = timed_kernel_loop(bwd, args.steps, args.warmup, world, flush)
+    btimes, blaunches = timed_kernel_loop(bwd, args.steps, args.warmup, world, flush, label="backward")
     bst = time_stats(btimes)
     bms_max = max_over_ranks(bst["mean"], world)
     b_flops = 2.5 * flops
@@ -557,7 +588,7 @@ def run_ours(args, world, rank, local):
     def merge():
         ea.attn_merge(mo_parts, ml_parts, o=m_out, lse=m_lse)
 
-    mtimes, mlaunches = timed_kernel_loop(merge, args.steps, args.warmup, world, None)
+    mtimes, mlaunches = timed_kernel_loop(merge, args.steps, args.warmup, world, None, label="merge")
     mst = time_stats(mtimes)
     mms_max = max_over_ranks(mst["mean"], world)
     m_rows = mw.B * mw.Nq * mw.Hq
@@ -586,7 +617,7 @@ def run_ours(args, world, rank, local):
     def fwd_varlen():
         ea.attn_fwd_varlen(vq, vk, vv, vcq, vck, vmax, vmax, o=vo, lse=vlse, causal=True)
 
-    vtimes, vlaunches = timed_kernel_loop(fwd_varlen, args.steps, args.warmup, world, flush)
+    vtimes, vlaunches = timed_kernel_loop(fwd_varlen, args.steps, args.warmup, world, flush, label="varlen")
     vst = time_stats(vtimes)
     vms_max = max_over_ranks(vst["mean"], world)
     v_flops = sum(metrics.attn_flops(1, 32, n, n, 128, True, -1) for n in vl_lens)
@@ -617,7 +648,7 @@ def run_ours(args, world, rank, local):
         ea.attn_decode(qd, kc, vc, o=od, lse=lsed, num_splits=args.decode_splits, workspace=ws)
 
     # the cache (2.1 GB) is far larger than L2, so no flush between decode steps
-    dtimes, dlaunches = timed_kernel_loop(dec, args.steps, args.warmup, world, None)
+    dtimes, dlaunches = timed_kernel_loop(dec, args.steps, args.warmup, world, None, label="decode")
     dst = time_stats(dtimes)
     dms_max = max_over_ranks(dst["mean"], world)
     kv_bytes = metrics.decode_kv_bytes([dw.Nk] * dw.B, dw.Hkv, dw.d)
@@ -651,7 +682,7 @@ def run_ours(args, world, rank, local):
         ea.attn_decode_paged(qd, kpg, vpg, bt, o=od, lse=lsed, num_splits=args.decode_splits,
                              workspace=ws)
 
-    ptimes, plaunches = timed_kernel_loop(dec_paged, args.steps, args.warmup, world, None)
+    ptimes, plaunches = timed_kernel_loop(dec_paged, args.steps, args.warmup, world, None, label="decode_paged")
     pst = time_stats(ptimes)
     pms_max = max_over_ranks(pst["mean"], world)
     decode_paged = {

@@ -160,6 +160,18 @@ struct Packed {
   int total_q, total_k;
 };
 
+// Multiplier and shift of attn::fdiv for the divisor d >= 1 (see FastDiv).
+attn::FastDiv make_fastdiv(int d) {
+  attn::FastDiv f{0u, 0u};
+  if (d <= 1) return f;
+  int l = 0;
+  while ((1ll << l) < d) ++l;                            // ceil(log2 d)
+  const unsigned long long two_p = 1ull << (31 + l);
+  f.m = static_cast<uint32_t>((two_p + static_cast<unsigned long long>(d) - 1) / static_cast<unsigned long long>(d));
+  f.s = static_cast<uint32_t>(l - 1);
+  return f;
+}
+
 template <int D, bool F32OUT, bool VARLEN>
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                int Hkv, int Nq, int Nk, float scale, int causal, int window_left,
@@ -239,6 +251,10 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
       if (kv_heads * kv_per_seq_head <= 96.0 * (1 << 20)) break;
     }
   }
+  p.fd_hg = make_fastdiv(p.hg);
+  p.fd_vlhg = make_fastdiv(p.vl_hg);
+  p.fd_per_b = make_fastdiv(p.nbh_seq);
+  p.fd_inner = make_fastdiv(p.pair_heads ? G / 2 : G);
   const long long items = static_cast<long long>(p.n_units) * p.n_bh;
   if (items > kMaxIndex) return fail(ATTN_ERR_INVALID_ARG, "problem too large for one launch");
   if (pk && (B > L::VL_MAX_SEQS || p.n_units > L::VL_MAX_UNITS))

@@ -107,6 +107,18 @@ struct FwdLayout {
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, 1);
 };
 
+// Division by a launch constant d without a divide: for 0 <= n < 2^31,
+// n / d = umulhi(n, m) >> s with l = ceil(log2 d), m = ceil(2^(31 + l) / d) and
+// s = l - 1 (Granlund and Montgomery, "Division by invariant integers using
+// multiplication", 1994); m = 0 stands for d = 1.
+struct FastDiv {
+  uint32_t m, s;
+};
+
+__device__ __forceinline__ int fdiv(int n, FastDiv f) {
+  return f.m ? int(__umulhi(uint32_t(n), f.m) >> f.s) : n;
+}
+
 struct FwdParams {
   void* o;                 // [B, Nq, Hq, D] bf16 or f32 (packed: [total_q, Hq, D])
   float* lse;              // [B, Hq, Nq] or null (packed: [Hq, total_q])
@@ -129,6 +141,9 @@ struct FwdParams {
   int hg;                  // equal lengths: (b, head-or-pair) per head group, divides n_bh
   int per_group;           // n_units * hg: items of one head group
   int bulk_o;              // equal-length bf16 O: 1 = staged bulk tensor stores, 0 = row stores
+  // divisors of the item decode: hg, vl_hg, the (b, head-or-pair) combinations
+  // per batch entry (Hkv * G/2 or Hq), and G/2 or G
+  FastDiv fd_hg, fd_vlhg, fd_per_b, fd_inner;
 };
 
 constexpr int kFwdThreads = 384;
@@ -295,16 +310,14 @@ __device__ void build_varlen_sched(const FwdParams& p, int* vl, int* n_items) {
 
 // vl: the packed-sequence tables (null for the closed-form work list).
 template <bool VARLEN>
-__device__ __forceinline__ void decode_item(const FwdParams& p, int item, WorkItem& w,
+__device__ __forceinline__ void decode_item(const FwdParams& p, int g, int ig, WorkItem& w,
                                             const int* vl) {
+  // item ig of head group g
   int unit, bh;
   if constexpr (VARLEN) {
     const int* lvl = vl + kVlLvl;
-    // head group, then level: the lowest u whose first item is <= the item's
-    // index within the group (lvl grows as u falls)
-    const int per_group = lvl[p.n_units];
-    const int g = item / per_group;
-    const int ig = item - g * per_group;
+    // level: the lowest u whose first item is <= the item's index within the
+    // group (lvl grows as u falls)
     int lo = 0, hi = p.n_units - 1;
     while (lo < hi) {
       const int mid = (lo + hi) >> 1;
@@ -312,33 +325,31 @@ __device__ __forceinline__ void decode_item(const FwdParams& p, int item, WorkIt
     }
     unit = lo;
     const int r = ig - lvl[unit];
-    const int s = r / p.vl_hg;
+    const int s = fdiv(r, p.fd_vlhg);
     bh = vl[s] * p.nbh_seq + g * p.vl_hg + (r - s * p.vl_hg);
   } else {
     // head groups one after another (so the K/V the running items touch stays
     // in L2), the longest rows first within a group
-    const int g = item / p.per_group;
-    const int ig = item - g * p.per_group;
-    const int lvl = ig / p.hg;
+    const int lvl = fdiv(ig, p.fd_hg);
     unit = p.n_units - 1 - lvl;
     bh = g * p.hg + (ig - lvl * p.hg);
   }
   if (p.pair_heads) {
     const int G = p.Hq / p.Hkv;
     const int pairs = G / 2;
-    w.b = bh / (p.Hkv * pairs);
-    const int rem = bh % (p.Hkv * pairs);
-    w.hkv = rem / pairs;
-    const int pr = rem % pairs;
+    w.b = fdiv(bh, p.fd_per_b);
+    const int rem = bh - w.b * (p.Hkv * pairs);
+    w.hkv = fdiv(rem, p.fd_inner);
+    const int pr = rem - w.hkv * pairs;
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
       w.tile[t].hq = w.hkv * G + 2 * pr + t;
       w.tile[t].row0 = unit * 128;
     }
   } else {
-    w.b = bh / p.Hq;
-    const int hq = bh % p.Hq;
-    w.hkv = hq / (p.Hq / p.Hkv);
+    w.b = fdiv(bh, p.fd_per_b);
+    const int hq = bh - w.b * p.Hq;
+    w.hkv = fdiv(hq, p.fd_inner);
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
       w.tile[t].hq = hq;
@@ -389,21 +400,25 @@ __device__ __forceinline__ void decode_item(const FwdParams& p, int item, WorkIt
 // CTAs. With one group this is the plain boustrophedon over the whole list.
 struct ItemCursor {
   int g = 0, k = 0;                        // group, this CTA's position within it
+  int start = 0;                           // first CTA of group g: g * per_group mod grid
 };
 
-__device__ __forceinline__ int next_item(ItemCursor& cur, int per_group, int n_groups) {
+// The index within group cur.g of this CTA's next item, or -1 when none is
+// left. pg_mod = per_group mod the grid size.
+__device__ __forceinline__ int next_item(ItemCursor& cur, int per_group, int n_groups, int pg_mod) {
   const int G = int(gridDim.x);
   while (cur.g < n_groups) {
-    const int start = int((static_cast<long long>(cur.g) * per_group) % G);
-    const int c0 = int(blockIdx.x) - start;
+    const int c0 = int(blockIdx.x) - cur.start;
     const int c = c0 < 0 ? c0 + G : c0;
     const long long i = static_cast<long long>(cur.k) * G + ((cur.k & 1) ? G - 1 - c : c);
     if (i < per_group) {
       ++cur.k;
-      return int(static_cast<long long>(cur.g) * per_group + i);
+      return int(i);
     }
     ++cur.g;
     cur.k = 0;
+    cur.start += pg_mod;
+    if (cur.start >= G) cur.start -= G;
   }
   return -1;
 }
@@ -473,6 +488,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     per_group = vl[kVlLvl + p.n_units];                 // items of one head group
     n_groups = p.nbh_seq / p.vl_hg;
   }
+  const int pg_mod = per_group % int(gridDim.x);
 
   if (warp < 8) {
     // ======================= softmax warpgroups ==============================
@@ -487,10 +503,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     bool ok = true;
     ItemCursor cur;
     while (ok) {
-      const int item = next_item(cur, per_group, n_groups);
-      if (item < 0) break;
+      const int ig = next_item(cur, per_group, n_groups, pg_mod);
+      if (ig < 0) break;
       WorkItem w;
-      decode_item<VARLEN>(p, item, w, vs);
+      decode_item<VARLEN>(p, cur.g, ig, w, vs);
       const TileInfo T = t ? w.tile[1] : w.tile[0];   // by value: no local-memory copy of w
       if (!T.active) continue;
       const int r = T.row0 + row;
@@ -742,10 +758,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       bool alive = true;
       ItemCursor cur;
       while (alive) {
-        const int item = next_item(cur, per_group, n_groups);
-        if (item < 0) break;
+        const int ig = next_item(cur, per_group, n_groups, pg_mod);
+        if (ig < 0) break;
         WorkItem w;
-        decode_item<VARLEN>(p, item, w, vs);
+        decode_item<VARLEN>(p, cur.g, ig, w, vs);
         if (w.U == 0) continue;
         if (!(alive = wwait(L::B_Q, uint32_t(qi & 1)))) break;
         tc_fence_after();
@@ -810,10 +826,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       bool alive = true;
       ItemCursor cur;
       while (alive) {
-        const int item = next_item(cur, per_group, n_groups);
-        if (item < 0) break;
+        const int ig = next_item(cur, per_group, n_groups, pg_mod);
+        if (ig < 0) break;
         WorkItem w;
-        decode_item<VARLEN>(p, item, w, vs);
+        decode_item<VARLEN>(p, cur.g, ig, w, vs);
         if (w.U == 0) continue;
         // Q buffers are free once every Q.K^T of the previous item completed
         if (qi > 0 && !(alive = mbar_wait(bar(L::B_QE), uint32_t((qi - 1) & 1), abort_flag))) break;
