@@ -539,9 +539,25 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           int lo = 0;
           if (p.window_left >= 0) lo = qpos - p.window_left;
           const int lo_rel = lo - kb0, hi_rel = hi - kb0;
+          // 32-key chunks that every row of the warp may see in full skip the
+          // compares (the choice is warp-uniform); on a causal diagonal block
+          // warp w has w such chunks.
+          const int lo_max = __reduce_max_sync(0xffffffffu, lo_rel);
+          const int hi_min = __reduce_min_sync(0xffffffffu, hi_rel);
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (c < lo_rel || c > hi_rel) s[c] = -CUDART_INF_F;
+          for (int q = 0; q < 4; ++q) {
+            if (32 * q < lo_max || 32 * q + 31 > hi_min) {
+              if (p.window_left >= 0) {
+#pragma unroll
+                for (int c = 32 * q; c < 32 * q + 32; ++c)
+                  if (c < lo_rel || c > hi_rel) s[c] = -CUDART_INF_F;
+              } else {                        // no window: lo_rel <= 0
+#pragma unroll
+                for (int c = 32 * q; c < 32 * q + 32; ++c)
+                  if (c > hi_rel) s[c] = -CUDART_INF_F;
+              }
+            }
+          }
         }
         // row max: 8 independent chains of three-input maxima
         float mx[8];
