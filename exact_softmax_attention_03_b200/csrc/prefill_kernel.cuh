@@ -24,11 +24,15 @@
 //   warps 10-11 idle (register budget only)
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D), O1 after it.
 // P_t is written as bf16 pairs over the first 64 columns of S_t and read by
-// the P·V product straight from TMEM.
+// the P·V product straight from TMEM. At the end of an item the softmax warps
+// store LSE, read O out of TMEM and write O / l: the equal-length bf16 kernel
+// through per-warp shared-memory blocks and bulk tensor stores, the others
+// row by row from registers.
 //
 // Masks ("Modern Attention ...", section 4 for the window; bottom-right causal
 // alignment): key blocks wholly outside a tile's allowed range are skipped;
-// boundary blocks are masked element by element in the softmax warps.
+// in boundary blocks the softmax warps compare element by element in the
+// 32-key chunks that some row of the warp may not see in full.
 // Every mbarrier wait is bounded (sm100_ptx.cuh); on a timeout the CTA stops
 // issuing work, drains what it issued, frees TMEM and exits.
 #pragma once
@@ -646,6 +650,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       if (!ok) break;
 
       // ---- epilogue: O / l and LSE -----------------------------------------
+      // LSE first: it needs only m and l, so its store overlaps the wait for
+      // the last P.V
+      const long long o_rows = VARLEN ? p.total_q : static_cast<long long>(p.B) * p.Nq;
+      const bool row_ok = r < T.nq &&
+                          in_bounds(VARLEN ? w.q0 + r : static_cast<long long>(w.b) * p.Nq + r, o_rows) &&
+                          in_bounds(T.hq, p.Hq);
+      if (row_ok && p.lse != nullptr) {
+        const size_t li = VARLEN ? size_t(T.hq) * p.total_q + w.q0 + r : (size_t(w.b) * p.Hq + T.hq) * p.Nq + r;
+        if (in_bounds(static_cast<long long>(li), static_cast<long long>(p.Hq) * o_rows))
+          p.lse[li] = (l > 0.f) ? fmaf(m, p.scale, __log2f(l) * 0.6931471805599453f) : -CUDART_INF_F;
+      }
       bool have = n_in_item > 0;
       if (have) {
         const bool wt = mbar_wait<1>(bar(L::B_OD + t), uint32_t((count - 1) & 1), abort_flag);
@@ -664,7 +679,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
         for (int e = 0; e < D; ++e) o[e] = 0u;
       }
-      const long long o_rows = VARLEN ? p.total_q : static_cast<long long>(p.B) * p.Nq;
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
       const bool bulk_o = kTmaO && p.bulk_o;
       if (bulk_o) {
@@ -700,8 +714,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           }
         }
       }
-      if (r < T.nq && in_bounds(VARLEN ? w.q0 + r : static_cast<long long>(w.b) * p.Nq + r, o_rows) &&
-          in_bounds(T.hq, p.Hq)) {
+      if (row_ok) {
         const size_t orow = VARLEN ? size_t(w.q0) + r : size_t(w.b) * p.Nq + r;
         const size_t obase = (orow * p.Hq + T.hq) * D;
         if constexpr (F32OUT) {
@@ -722,9 +735,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             dst[e] = v;
           }
         }
-        const size_t li = VARLEN ? size_t(T.hq) * p.total_q + w.q0 + r : (size_t(w.b) * p.Hq + T.hq) * p.Nq + r;
-        if (p.lse != nullptr && in_bounds(static_cast<long long>(li), static_cast<long long>(p.Hq) * o_rows))
-          p.lse[li] = (l > 0.f) ? fmaf(m, p.scale, __log2f(l) * 0.6931471805599453f) : -CUDART_INF_F;
       }
     }
     // the CTA's shared memory must outlive the last O stores
