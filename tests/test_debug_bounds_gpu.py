@@ -7,7 +7,7 @@ is reported by attn_device_status() as ATTN_ERR_INTERNAL. It stands in for a
 memory checker, which cannot run on these machines.
 
 Here the small forward (plain, windowed, GQA, packed), decode (contiguous and
-paged), backward and merge parity tests run in a child process against the
+paged), backward, merge and random-shape parity tests run in a child process against the
 debug build (ATTN_LIBRARY=debug): every call must pass parity with the fp64
 oracle and leave the status word clear. So does the full-size MHA causal
 N = 8192 forward, the one workload here whose work list runs in head groups.
@@ -35,6 +35,7 @@ CASES = [
     "tests/test_decode_paged_gpu.py",
     "tests/test_bwd_gpu.py",
     "tests/test_context_parallel_gpu.py",
+    "tests/test_random_shapes_gpu.py",
 ]
 
 
