@@ -56,17 +56,22 @@ def build(force: bool = False, verbose: bool = False, debug: bool | None = None)
     lib = LIB_DEBUG if debug else LIB
     if not force and up_to_date(lib):
         return lib
-    cmd = [nvcc_path(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-o", lib + ".tmp", SRC]
+    # a private temporary name: ranks of one job that build at once each write
+    # their own file, and the atomic rename leaves one complete library
+    tmp = f"{lib}.{os.getpid()}.tmp"
+    cmd = [nvcc_path(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-o", tmp, SRC]
     if debug:
         cmd += ["-DATTN_DEBUG_BOUNDS=1"]
     if verbose:
         cmd += ["-Xptxas", "-v"]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
+        if os.path.exists(tmp):
+            os.remove(tmp)
         raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + res.stdout + res.stderr)
     if verbose:
         sys.stderr.write(res.stdout + res.stderr)
-    os.replace(lib + ".tmp", lib)
+    os.replace(tmp, lib)
     return lib
 
 
