@@ -96,15 +96,18 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 // {64, 1, 128, 1} with 128-byte swizzle (one 128-row x 128-byte block).
 // 4-D view {d, H, N, B} of a [B, N, H, d] bf16 tensor, boxes of 64 columns x
 // box_rows rows with the 128-byte swizzle.
-int make_map(CUtensorMap* map, const void* base, int d, int H, int N, int B, int box_rows = 128) {
+// (box_cols = 32: 64-byte rows with the 64-byte swizzle.)
+int make_map(CUtensorMap* map, const void* base, int d, int H, int N, int B, int box_rows = 128,
+             int box_cols = 64) {
   auto enc = tensor_map_encoder();
   if (enc == nullptr) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   cuuint64_t dims[4] = {cuuint64_t(d), cuuint64_t(H), cuuint64_t(N), cuuint64_t(B)};
   cuuint64_t strides[3] = {cuuint64_t(d) * 2, cuuint64_t(H) * d * 2, cuuint64_t(N) * H * d * 2};
-  cuuint32_t box[4] = {64, 1, cuuint32_t(box_rows), 1};
+  cuuint32_t box[4] = {cuuint32_t(box_cols), 1, cuuint32_t(box_rows), 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   box_cols == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
   return ATTN_OK;
@@ -184,8 +187,10 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   if ((rc = make_map(&mq, q, D, Hq, rq, nb)) != ATTN_OK) return rc;
   if ((rc = make_map(&mk, k, D, Hkv, rk, nb)) != ATTN_OK) return rc;
   if ((rc = make_map(&mv, v, D, Hkv, rk, nb)) != ATTN_OK) return rc;
-  CUtensorMap mo = mq;                 // O map: used by the equal-length bf16 kernel only
-  if (!VARLEN && !F32OUT && (rc = make_map(&mo, o, D, Hq, Nq, B, 32)) != ATTN_OK) return rc;
+  CUtensorMap mo = mq;                 // O map: used by the bf16-output kernels only
+  if (!F32OUT && (rc = (VARLEN ? make_map(&mo, o, D, Hq, rq, 1, 32, 32)
+                               : make_map(&mo, o, D, Hq, Nq, B, 32))) != ATTN_OK)
+    return rc;
 
   attn::FwdParams p{};
   p.o = o;
@@ -234,9 +239,9 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     }
   }
   p.per_group = p.n_units * p.hg;
-  // equal-length bf16 O: staged bulk tensor stores (the kernel keeps the
-  // per-row stores as a launch-time alternative, p.bulk_o = 0)
-  p.bulk_o = (!pk && !F32OUT) ? 1 : 0;
+  // bf16 O: staged bulk tensor stores (the kernel keeps the per-row stores as a
+  // launch-time alternative, p.bulk_o = 0)
+  p.bulk_o = !F32OUT ? 1 : 0;
   if (pk) {
     // Head groups for the packed work list: the largest divisor of the items per
     // (sequence, unit) for which the K/V the concurrently running items touch

@@ -45,14 +45,15 @@
 namespace attn {
 
 // Packed-sequence schedule tables in shared memory (ints): perm[kVlMaxSeqs]
-// (sequences sorted by row units, longest first), cnt[kVlMaxUnits + 1]
-// (cnt[u]: sequences with more than u units), lvl[kVlMaxUnits + 1] (first
-// item of unit level u), cur[kVlMaxUnits + 1] (scatter cursors).
+// (sequences sorted by row units, longest first), lvl[kVlMaxUnits + 1] (first
+// item of unit level u), cnt[kVlMaxUnits + 1] (cnt[u]: sequences with more
+// than u units), cur[kVlMaxUnits + 1] (scatter cursors). cnt and cur serve
+// only the build at kernel start; their space then holds O staging blocks.
 constexpr int kVlMaxSeqs = 2048;
 constexpr int kVlMaxUnits = 1024;
-constexpr int kVlCnt = kVlMaxSeqs;
-constexpr int kVlLvl = kVlCnt + kVlMaxUnits + 1;
-constexpr int kVlCur = kVlLvl + kVlMaxUnits + 1;
+constexpr int kVlLvl = kVlMaxSeqs;
+constexpr int kVlCnt = kVlLvl + kVlMaxUnits + 1;
+constexpr int kVlCur = kVlCnt + kVlMaxUnits + 1;
 constexpr int kVlInts = kVlCur + kVlMaxUnits + 1;
 
 #ifndef ATTN_VSTAGES
@@ -103,7 +104,12 @@ struct FwdLayout {
   static constexpr int VL_MAX_SEQS = kVlMaxSeqs;
   static constexpr int VL_MAX_UNITS = kVlMaxUnits;
   static constexpr int OFF_VL = OFF_DBG + 32;                            // VarlenTables
-  static constexpr int BYTES = OFF_VL + (VARLEN ? 4 * kVlInts : 0);
+  // packed kernel: a 32-row x 32-column O staging block (2 KB) per softmax
+  // warp, over the schedule tables' build-time part (cnt, cur) and beyond
+  static constexpr int OFF_OSTV = (OFF_VL + 4 * kVlCnt + 1023) / 1024 * 1024;
+  static constexpr int BYTES_VL = OFF_VL + 4 * kVlInts > OFF_OSTV + 8 * 2048
+                                      ? OFF_VL + 4 * kVlInts : OFF_OSTV + 8 * 2048;
+  static constexpr int BYTES = VARLEN ? BYTES_VL : OFF_VL;
   static constexpr int SMEM_ALLOC = BYTES + 1024;       // slack for 1024-byte alignment
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
@@ -439,6 +445,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   // stays a launch parameter: built that way, the kernel measured 1-3 points
   // of the bf16 peak faster than with the bulk stores fixed at compile time.
   constexpr bool kTmaO = !VARLEN && !F32OUT;
+  // the packed kernel stores O the same way from the warps whose 32 rows all
+  // lie inside their sequence, through 2 KB blocks of 32 columns
+  constexpr bool kTmaOV = VARLEN && !F32OUT;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -680,16 +689,46 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         for (int e = 0; e < D; ++e) o[e] = 0u;
       }
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
-      const bool bulk_o = kTmaO && p.bulk_o;
-      if (bulk_o) {
+      const bool bulk_o = (kTmaO || kTmaOV) && p.bulk_o;
+      const int wr0 = T.row0 + 32 * (warp & 3);
+      const bool warp_bulk = bulk_o && (VARLEN ? wr0 + 32 <= T.nq : wr0 < T.nq);
+      if constexpr (kTmaOV) {
+        if (warp_bulk) {
+          // 32 columns at a time: 64-byte rows with the 64-byte swizzle of the
+          // tensor map; the block is rewritten after its previous store read it
+          const uint32_t stg = sb + L::OFF_OSTV + uint32_t(warp) * 2048u;
+          const uint32_t rb = stg + uint32_t(lane) * 64u;
+#pragma unroll
+          for (int qc = 0; qc < D / 32; ++qc) {
+            if (lane == 0) bulk_wait_read_all();
+            __syncwarp();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const uint32_t* e = o + 32 * qc + 8 * c;
+              st_shared_v4(rb + uint32_t((c ^ ((lane >> 1) & 3)) << 4),
+                           pack_bf16x2(__uint_as_float(e[0]) * inv, __uint_as_float(e[1]) * inv),
+                           pack_bf16x2(__uint_as_float(e[2]) * inv, __uint_as_float(e[3]) * inv),
+                           pack_bf16x2(__uint_as_float(e[4]) * inv, __uint_as_float(e[5]) * inv),
+                           pack_bf16x2(__uint_as_float(e[6]) * inv, __uint_as_float(e[7]) * inv));
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && in_bounds(T.hq, p.Hq) &&
+                in_bounds(static_cast<long long>(w.q0) + wr0 + 31, static_cast<long long>(p.total_q))) {
+              tma_store_4d(&tmO, stg, 32 * qc, T.hq, w.q0 + wr0, 0);
+              bulk_commit_group();
+            }
+          }
+        }
+      }
+      if (kTmaO && warp_bulk) {
         // Each warp writes its 32 rows to its own staging block, 64 columns at
         // a time, in the 128-byte swizzled layout of the tensor map; lane 0
         // then stores the block (rows past Nq fall outside the map and are not
         // written). A block is rewritten only after its previous store has
         // read it. Only warp-level synchronisation: no warp ever waits on
         // another one here.
-        const int wr0 = T.row0 + 32 * (warp & 3);
-        if (wr0 < T.nq) {
+        {
           const uint32_t stg = sb + L::OFF_OST + uint32_t(t) * L::HALF + uint32_t(warp & 3) * 4096u;
           const uint32_t rbase = stg + uint32_t(lane) * 128u;
 #pragma unroll
@@ -723,7 +762,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           for (int e = 0; e < D / 4; ++e)
             dst[e] = make_float4(__uint_as_float(o[4 * e]) * inv, __uint_as_float(o[4 * e + 1]) * inv,
                                  __uint_as_float(o[4 * e + 2]) * inv, __uint_as_float(o[4 * e + 3]) * inv);
-        } else if (!bulk_o) {
+        } else if (!warp_bulk) {
           uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) + obase);
 #pragma unroll
           for (int e = 0; e < D / 8; ++e) {
@@ -738,7 +777,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
     }
     // the CTA's shared memory must outlive the last O stores
-    if (kTmaO && lane == 0) bulk_wait_all();
+    if ((kTmaO || kTmaOV) && lane == 0) bulk_wait_all();
     if (row == 0) reinterpret_cast<volatile int*>(smem + L::OFF_DBG)[4 + t] = count;
   } else {
   // warps 8-11 release registers to the softmax warpgroups (the release is
