@@ -25,9 +25,10 @@
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D), O1 after it.
 // P_t is written as bf16 pairs over the first 64 columns of S_t and read by
 // the P·V product straight from TMEM. At the end of an item the softmax warps
-// store LSE, read O out of TMEM and write O / l: the equal-length bf16 kernel
-// through per-warp shared-memory blocks and bulk tensor stores, the others
-// row by row from registers.
+// store LSE, read O out of TMEM and write O / l: bf16 O through per-warp
+// shared-memory blocks and bulk tensor stores (in the packed kernel from the
+// warps whose rows all lie inside their sequence), the rest row by row from
+// registers.
 //
 // Masks ("Modern Attention ...", section 4 for the window; bottom-right causal
 // alignment): key blocks wholly outside a tile's allowed range are skipped;
@@ -440,7 +441,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 const FwdParams p) {
   using L = FwdLayout<D, VARLEN>;
   // bf16 O of the equal-length kernel leaves through shared memory and bulk
-  // tensor stores (tmO) when p.bulk_o, which the host sets for every such
+  // tensor stores (tmO) when p.bulk_o, which the host sets for every bf16
   // launch; otherwise each thread stores its row from registers. The choice
   // stays a launch parameter: built that way, the kernel measured 1-3 points
   // of the bf16 peak faster than with the bulk stores fixed at compile time.
