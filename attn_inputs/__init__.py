@@ -7,7 +7,9 @@ checks may use it without sharing any of the method.
 Recipe: one CPU ``torch.Generator`` per tensor, seeded ``seed``, ``seed + 1``,
 ``seed + 2`` for q, k, v; ``randn`` in float32 (iid N(0, 1)), then rounded to
 bfloat16 on the host. The identical bf16 tensors go to the GPU and, upcast
-exactly, to the oracle.
+exactly, to the oracle. The ``*_on`` variants draw the same way with a
+generator on the given device (torch's own random numbers, none of this
+library's kernels); the oracle then reads back the slices it checks.
 """
 
 from __future__ import annotations
@@ -77,9 +79,38 @@ def make_decode(B, Hq, Hkv, Lmax, d, seed: int = SEED_Q):
     return q, k, v
 
 
+def _randn_on(shape, seed: int, device) -> torch.Tensor:
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    return torch.randn(*shape, generator=g, dtype=torch.float32, device=device).to(torch.bfloat16)
+
+
+def make_qkv_on(device, B, Hq, Hkv, Nq, Nk, d, seed: int = SEED_Q):
+    """As :func:`make_qkv`, but drawn by a torch generator on ``device``: for
+    tensors of several GB, which the host would take long to draw and copy.
+    Same distribution (iid N(0, 1) rounded to bf16); other values."""
+    q = _randn_on((B, Nq, Hq, d), seed, device)
+    k = _randn_on((B, Nk, Hkv, d), seed + 1, device)
+    v = _randn_on((B, Nk, Hkv, d), seed + 2, device)
+    return q, k, v
+
+
+def make_decode_on(device, B, Hq, Hkv, Lmax, d, seed: int = SEED_Q):
+    """As :func:`make_decode`, drawn on ``device`` (see :func:`make_qkv_on`)."""
+    q = _randn_on((B, Hq, d), seed, device)
+    k = _randn_on((B, Lmax, Hkv, d), seed + 1, device)
+    v = _randn_on((B, Lmax, Hkv, d), seed + 2, device)
+    return q, k, v
+
+
 def make_dout(B, Nq, Hq, d, seed: int = SEED_Q + 21):
     """bf16 CPU upstream gradient ``dO [B, Nq, Hq, d]`` (iid normal)."""
     return _randn((B, Nq, Hq, d), seed)
+
+
+def make_dout_on(device, B, Nq, Hq, d, seed: int = SEED_Q + 21):
+    """As :func:`make_dout`, drawn on ``device`` (see :func:`make_qkv_on`)."""
+    return _randn_on((B, Nq, Hq, d), seed, device)
 
 
 def make_for(w: Workload, seed: int = SEED_Q):

@@ -117,3 +117,39 @@ def test_full_size_sampled_groups(shape, causal, wl):
         ref = backward_of_group(q, k, v, do, b, hk, causal, wl)
         got = (dq[b, :, hk * G:(hk + 1) * G], dk[b, :, hk], dv[b, :, hk])
         compare(got, ref, (shape, causal, wl, b, hk))
+
+
+def test_tensors_past_4_gib():
+    """Q, K, V, O, dO and the three gradients of 4.56 GB each (B1 N131072 H136
+    d128: more than 2^31 elements, byte offsets past 2^32), causal with a
+    window of 128 keys. With that window a span of rows and keys is a closed
+    problem away from its edges: the oracle's backward of the span gives the
+    exact dQ of its rows that see 128 keys inside it and the exact dK, dV of
+    its keys whose 128 queries lie inside it. Spans at the start, in the middle
+    and at the end (past 2^32 bytes) of two heads are compared."""
+    import exact_softmax_attention_03_b200 as ea
+    B, H, N, d, wl, S = 1, 136, 131072, 128, 127, 1024
+    q, k, v = ai.make_qkv_on("cuda", B, H, H, N, N, d, seed=ai.SEED_Q + 62)
+    do = ai.make_dout_on("cuda", B, N, H, d, seed=ai.SEED_Q + 63)
+    assert q.numel() > 2 ** 31 and q.numel() * q.element_size() > 2 ** 32
+    lse = torch.empty(B, H, N, device="cuda")
+    o, _ = ea.attn_fwd(q, k, v, lse=lse, causal=True, window_left=wl)
+    dq, dk, dv = ea.attn_bwd(q, k, v, o, lse, do, causal=True, window_left=wl)
+    assert ea.attn_device_status() == 0
+    for t in (dq, dk, dv):
+        assert torch.isfinite(t).all()
+    del o
+    for h in (0, H - 1):
+        for s0 in (0, N // 2 - S // 2, N - S):
+            s1 = s0 + S
+            sl = (slice(0, 1), slice(s0, s1), slice(h, h + 1))
+            rq, rk, rv = oracle.oracle_attention_backward(q[sl].cpu(), k[sl].cpu(), v[sl].cpu(),
+                                                          do[sl].cpu(), causal=True, window_left=wl)
+            r_lo = s0 if s0 == 0 else s0 + wl                 # rows whose keys lie in the span
+            k_lo = s0 if s0 == 0 else s0 + wl                 # keys whose queries' sums are exact
+            k_hi = s1 if s1 == N else s1 - wl                 # keys whose queries lie in the span
+            got = (dq[0, r_lo:s1, h], dk[0, k_lo:k_hi, h], dv[0, k_lo:k_hi, h])
+            ref = (rq[0, r_lo - s0:, 0], rk[0, k_lo - s0:k_hi - s0, 0], rv[0, k_lo - s0:k_hi - s0, 0])
+            compare(got, ref, ("past 4 GiB", h, s0))
+    del q, k, v, do, dq, dk, dv
+    torch.cuda.empty_cache()

@@ -102,3 +102,27 @@ def test_decode_caller_workspace_and_repeat():
     assert torch.equal(o1, o2)
     O, _ = oracle.oracle_decode(q, kc, vc)
     assert_close(o1, O)
+
+
+def test_caches_past_4_gib():
+    """K and V caches of 4.56 GB each (B4 Lmax131072 Hkv34 d128: more than
+    2^31 elements, byte offsets past 2^32), Hq 136 (groups of 4), ragged
+    lengths with the last sequence full, so the last keys read lie past 2^32
+    bytes. Eight query heads of every sequence are compared with the oracle."""
+    import exact_softmax_attention_03_b200 as ea
+    B, Hq, Hkv, L, d = 4, 136, 34, 131072, 128
+    q, kc, vc = ai.make_decode_on("cuda", B, Hq, Hkv, L, d, seed=ai.SEED_Q + 61)
+    assert kc.numel() > 2 ** 31 and kc.numel() * kc.element_size() > 2 ** 32
+    sl = torch.tensor([L, 77777, 1, L], dtype=torch.int32)
+    lse = torch.empty(B, Hq, device="cuda")
+    o, _ = ea.attn_decode(q, kc, vc, lse=lse, seqlens=sl.cuda())
+    assert ea.attn_device_status() == 0
+    G = Hq // Hkv
+    for b, h0 in ((0, 0), (1, 64), (2, 8), (3, Hq - 8)):
+        hs = slice(h0, h0 + 8)
+        ks = slice(h0 // G, (h0 + 8) // G)
+        O, Lr = oracle.oracle_decode(q[b:b + 1, hs].cpu(), kc[b:b + 1, :, ks].cpu(),
+                                     vc[b:b + 1, :, ks].cpu(), sl[b:b + 1])
+        assert_close(o[b:b + 1, hs], O, lse[b:b + 1, hs], Lr, what=("caches past 4 GiB", b, h0))
+    del q, kc, vc, o
+    torch.cuda.empty_cache()

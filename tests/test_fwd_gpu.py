@@ -216,3 +216,27 @@ def test_overflow_in_second_half_of_a_block():
         o, lse = run_fwd(q, k, v, causal, wl)
         O, L = oracle.oracle_attention(q, k, v, causal=causal, window_left=wl)
         assert_close(o, O, lse, L, what=("second half", causal, wl))
+
+
+def test_tensors_past_4_gib():
+    """Q, K, V and O of 4.56 GB each (B1 N131072 H136 d128: more than 2^31
+    elements, byte offsets past 2^32 in every tensor), causal with a window of
+    128 keys so the launch stays short. Rows at the start, in the middle and at
+    the end (past 2^32 bytes) of three heads are compared element by element
+    with the oracle; every output must be finite."""
+    import exact_softmax_attention_03_b200 as ea
+    B, H, N, d, wl = 1, 136, 131072, 128, 127
+    q, k, v = ai.make_qkv_on("cuda", B, H, H, N, N, d, seed=ai.SEED_Q + 60)
+    assert q.numel() > 2 ** 31 and q.numel() * q.element_size() > 2 ** 32
+    lse = torch.empty(B, H, N, device="cuda")
+    o, _ = ea.attn_fwd(q, k, v, lse=lse, causal=True, window_left=wl)
+    assert ea.attn_device_status() == 0
+    assert torch.isfinite(o).all() and torch.isfinite(lse).all()
+    rows = list(range(0, 64)) + list(range(N // 2 - 32, N // 2 + 32)) + list(range(N - 64, N))
+    for h in (0, 67, H - 1):
+        O, L = oracle.oracle_attention_rows(_head(q, 0, h).cpu(), _head(k, 0, h).cpu(),
+                                            _head(v, 0, h).cpu(), 0, 0, rows, causal=True,
+                                            window_left=wl)
+        assert_close(o[0, rows, h], O, lse[0, h, rows], L, what=("past 4 GiB", h))
+    del q, k, v, o
+    torch.cuda.empty_cache()
