@@ -17,20 +17,24 @@
 //                       accumulator with vector atomics
 //   bwd_finalize_kernel dQ accumulator -> bf16
 //
-// bwd_main_kernel warp roles (352 threads):
-//   warps 0-3  elementwise, thread = TMEM lane = key row: P, then dS, per
-//              block; at the end dK, dV
-//   warps 4-7  dQ, thread = TMEM lane = query row: read dQ_i out of tensor
+// bwd_main_kernel warp roles (480 threads):
+//   warps 0-7  elementwise, thread = TMEM lane = key row: P, then dS, per
+//              block; at the end dK, dV. Warps w and w + 4 share the key rows
+//              of lanes 32 (w % 4) .. + 31, warp w takes queries [0, 64) of a
+//              block and warp w + 4 queries [64, 128), so each SM
+//              sub-partition runs two of them
+//   warps 8-11 dQ, thread = TMEM lane = query row: read dQ_i out of tensor
 //              memory, add it to the accumulator
-//   warp 8     tensor-core issuer (whole warp, one elected lane issues)
-//   warp 9     TMA producer (one lane): K_j, V_j once; Q_i, dO_i per block
+//   warp 12    tensor-core issuer (whole warp, one elected lane issues)
+//   warp 13    TMA producer (one lane): K_j, V_j once; Q_i, dO_i per block
 //              through a 2-stage ring (the next block's tiles load during this one)
-//   warp 10    stages each block's lse2 / delta values in shared memory
+//   warp 14    stages each block's lse2 / delta values in shared memory
 // Per query block (tile = 128 x 128), TMEM cols [0,128) Sᵀ / Pᵀ, [128,256)
 // dPᵀ / dQ_i, [256,256+D) dV, [256+D,256+2D) dK:
 //   Sᵀ  = K_j Q_iᵀ        SS, both K-major (N = 128)
-//   phase P: Pᵀ = exp2(Sᵀ c - lse2) as bf16 pairs over cols [0,64); the pairs
-//     stay in registers
+//   phase P: Pᵀ = exp2(Sᵀ c - lse2) as bf16 pairs, queries [0,64) over cols
+//     [0,32) and queries [64,128) over cols [64,96) (each half over Sᵀ columns
+//     its own warps have read); the pairs stay in registers
 //   dV += Pᵀ dO_i         TS: A = Pᵀ (TMEM), B = dO_i MN-major
 //   dPᵀ = V_j dO_iᵀ       SS, both K-major (N = 128)
 //   phase dS: dSᵀ = Pᵀ (dPᵀ - delta) from those bf16 P, to shared memory only
@@ -229,7 +233,7 @@ struct BwdLayout {
   static constexpr uint32_t IDESC_DQ = idesc_bf16_f32_amn(128, D, 1);
 };
 
-constexpr int kBwdThreads = 352;
+constexpr int kBwdThreads = 480;
 
 // Query blocks that hold at least one allowed (query, key) pair with a key in
 // [kb0, kb1]: [i_lo, i_hi], empty when i_hi < i_lo.
@@ -286,8 +290,8 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
     mbar_init(bar(L::B_SS), 1);
     mbar_init(bar(L::B_SP), 1);
-    mbar_init(bar(L::B_PA), 128);
-    mbar_init(bar(L::B_PB), 128);
+    mbar_init(bar(L::B_PA), 256);
+    mbar_init(bar(L::B_PB), 256);
     mbar_init(bar(L::B_DVD), 1);
     mbar_init(bar(L::B_QR), 1);
     mbar_init(bar(L::B_QF), 128);
@@ -296,7 +300,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 8) {
+  if (warp == 12) {
     tmem_alloc(smem_u32(tmem_holder), L::TMEM_COLS);
     tmem_relinquish();
   }
@@ -305,10 +309,13 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp < 4) {
+  if (warp < 8) {
     // ======================= elementwise warps ==============================
-    const int t = int(threadIdx.x);                          // TMEM lane
-    const uint32_t lane_off = uint32_t(warp * 32) << 16;
+    // warps w and w + 4 share TMEM lanes 32 (w % 4) .. + 31 (their key rows);
+    // warp w takes queries [0, 64) of each block, warp w + 4 queries [64, 128)
+    const int t = int(threadIdx.x) & 127;                    // TMEM lane
+    const int hh = warp >> 2;                                // query half
+    const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
     const uint32_t tST = tmem + lane_off + L::COL_ST, tDPT = tmem + lane_off + L::COL_DPT;
     const float* lsr = reinterpret_cast<const float*>(smem + L::OFF_LD);   // lse2[128]
     const float* dlt = lsr + 128;                                           // delta[128]
@@ -328,12 +335,13 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       if (key >= p.Nk) c_hi = -1;
       if (p.causal) c_lo = max(c_lo, key - off - q0);                    // key <= q + off
       if (p.window_left >= 0) c_hi = min(c_hi, key + p.window_left - off - q0);
-      // phase A, 32 queries at a time: Pᵀ over columns of Sᵀ already read
-      // (chunk c -> columns [16c, 16c + 16)); the bf16 pairs stay in registers
-      uint32_t pw[4][16];
+      // phase A, 32 queries at a time: Pᵀ over columns of Sᵀ this warp has
+      // already read (queries [64h + 32c, +32) -> columns [64h + 16c, +16)); the
+      // bf16 pairs stay in registers
+      uint32_t pw[2][16];
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        const int c0 = 32 * cc;
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c0 = 64 * hh + 32 * cc;
         uint32_t sr[32];
         tmem_ld32(tST + c0, sr);
         tmem_wait_ld();
@@ -341,7 +349,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           bwd_p<false>(sr, lsr, c0, c_lo, c_hi, c2, pw[cc]);
         else
           bwd_p<true>(sr, lsr, c0, c_lo, c_hi, c2, pw[cc]);
-        tmem_st16(tST + 16 * cc, pw[cc]);
+        tmem_st16(tST + 64 * hh + 16 * cc, pw[cc]);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -351,18 +359,18 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(L::B_SP), par, abort_flag)))) break;
       tc_fence_after();
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        const int c0 = 32 * cc;
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c0 = 64 * hh + 32 * cc;
         uint32_t dr[32], dw[16];
         tmem_ld32(tDPT + c0, dr);
         tmem_wait_ld();
         bwd_ds(dr, pw[cc], dlt, c0, dw);
-        // dSᵀ row of this key -> shared memory block cc / 2 (queries 64h..64h+63),
+        // dSᵀ row of this key -> shared memory block hh (queries 64hh..64hh+63),
         // 16-byte chunks swizzled by (row & 7)
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
-          const int chunk = 4 * (cc & 1) + ch;
-          const uint32_t addr = sb + L::OFF_DS + (cc >> 1) * L::HALF + t * 128 + ((chunk ^ (t & 7)) * 16);
+          const int chunk = 4 * cc + ch;
+          const uint32_t addr = sb + L::OFF_DS + hh * L::HALF + t * 128 + ((chunk ^ (t & 7)) * 16);
           asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
                        ::"r"(addr), "r"(dw[4 * ch]), "r"(dw[4 * ch + 1]), "r"(dw[4 * ch + 2]),
                        "r"(dw[4 * ch + 3]) : "memory");
@@ -371,25 +379,26 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       tc_fence_before();
       mbar_arrive(bar(L::B_PB));
-      if (t == 0) reinterpret_cast<volatile int*>(smem + L::OFF_MISC)[3] = n + 1;
+      if (threadIdx.x == 0) reinterpret_cast<volatile int*>(smem + L::OFF_MISC)[3] = n + 1;
     }
     // ---- dK, dV of this key row ---------------------------------------------
     const bool have = ok && total > 0 &&
                       __all_sync(0xffffffffu, mbar_wait(bar(L::B_DONE), 0u, abort_flag));
     if (have) tc_fence_after();
-    // Each warp stages its 32 key rows of dV, then dK (scaled), as 4 KB blocks
-    // of 32 rows x 64 columns in the 128-byte swizzled layout of the tensor
-    // maps, in the Q ring (free once every product has completed); lane 0
-    // stores the blocks. Rows past Nk fall outside the maps and are not written.
-    const int wk0 = kb0 + 32 * warp;
-    if ((have || (ok && total == 0)) && wk0 < p.Nk) {
-      constexpr int NH = D / 64;
-      const uint32_t stg = sb + L::OFF_Q + uint32_t(warp) * (2 * NH * 4096);
+    // Each warp stages its 32 key rows of dV, then dK (scaled), for its
+    // 64-column half hh, as 4 KB blocks of 32 rows x 64 columns in the 128-byte
+    // swizzled layout of the tensor maps, in the Q ring (free once every product
+    // has completed); lane 0 stores the blocks. Rows past Nk fall outside the
+    // maps and are not written. At D = 64 the warps of half 0 do it all.
+    constexpr int NH = D / 64;
+    const int wk0 = kb0 + 32 * (warp & 3);
+    if ((have || (ok && total == 0)) && wk0 < p.Nk && hh < NH) {
+      const uint32_t stg = sb + L::OFF_Q + uint32_t(warp & 3) * (2 * NH * 4096);
 #pragma unroll
       for (int m = 0; m < 2; ++m) {                          // 0: dV, 1: dK (scaled)
         const float f = m ? p.scale : 1.f;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 2 * hh; c < 2 * hh + 2; ++c) {
           uint32_t r[32];
           if (have) {
             tmem_ld32(tmem + lane_off + (m ? L::COL_DK : L::COL_DV) + 32 * c, r);
@@ -413,41 +422,47 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       if (lane == 0 && in_bounds(b, p.B) && in_bounds(hkv, p.Hkv)) {
 #pragma unroll
         for (int m = 0; m < 2; ++m)
-#pragma unroll
-          for (int h = 0; h < NH; ++h)
-            tma_store_4d(m ? &tmDK : &tmDV, stg + uint32_t(m * NH + h) * 4096u, 64 * h, hkv, wk0, b);
+          tma_store_4d(m ? &tmDK : &tmDV, stg + uint32_t(m * NH + hh) * 4096u, 64 * hh, hkv, wk0, b);
         bulk_commit_group();
         bulk_wait_all();                    // shared memory outlives the stores
       }
     }
-  } else if (warp < 8) {
+  } else if (warp < 12) {
     // ======================= dQ warps ========================================
-    const int r = int(threadIdx.x) - 128;                    // TMEM lane = query row in the block
-    const uint32_t tDQ = tmem + (uint32_t((warp - 4) * 32) << 16) + L::COL_DPT;
+    const int r = int(threadIdx.x) - 256;                    // TMEM lane = query row in the block
+    const uint32_t tDQ = tmem + (uint32_t((warp - 8) * 32) << 16) + L::COL_DPT;
     for (int n = 0; n < total; ++n) {
       const int hq = hkv * G + n / nblk, q = (i_lo + n % nblk) * 128 + r;
       const uint32_t par = uint32_t(n & 1);
       if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_QR), par, abort_flag))) break;
       tc_fence_after();
-      uint32_t qr[D];
+      const bool qok = q < p.Nq && in_bounds((static_cast<long long>(b) * p.Hq + hq) * p.Nq + q,
+                                             static_cast<long long>(p.B) * p.Hq * p.Nq);
+      // chunk e of query q: the warp's 32 queries are 32 adjacent float4
+      float4* dst = reinterpret_cast<float4*>(p.dq_acc) + (size_t(b) * p.Hq + hq) * (D / 4) * p.Nq +
+                    (qok ? q : 0);
+      // 64 columns at a time (the register budget of 15 warps); the columns
+      // are released once the last ones are read
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) tmem_ld32(tDQ + 32 * c, qr + 32 * c);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bar(L::B_QF));
-      if (q < p.Nq && in_bounds((static_cast<long long>(b) * p.Hq + hq) * p.Nq + q,
-                                static_cast<long long>(p.B) * p.Hq * p.Nq)) {
-        // chunk e of query q: the warp's 32 queries are 32 adjacent float4
-        float4* dst = reinterpret_cast<float4*>(p.dq_acc) + (size_t(b) * p.Hq + hq) * (D / 4) * p.Nq + q;
+      for (int hf = 0; hf < D / 64; ++hf) {
+        uint32_t qr[64];
+        tmem_ld32(tDQ + 64 * hf, qr);
+        tmem_ld32(tDQ + 64 * hf + 32, qr + 32);
+        tmem_wait_ld();
+        if (hf == D / 64 - 1) {
+          tc_fence_before();
+          mbar_arrive(bar(L::B_QF));
+        }
+        if (qok) {
 #pragma unroll
-        for (int e = 0; e < D / 4; ++e)
-          atomicAdd(dst + size_t(e) * p.Nq, make_float4(__uint_as_float(qr[4 * e]) * p.scale,
-                                                        __uint_as_float(qr[4 * e + 1]) * p.scale,
-                                                        __uint_as_float(qr[4 * e + 2]) * p.scale,
-                                                        __uint_as_float(qr[4 * e + 3]) * p.scale));
+          for (int e = 0; e < 16; ++e)
+            atomicAdd(dst + size_t(16 * hf + e) * p.Nq,
+                      make_float4(__uint_as_float(qr[4 * e]) * p.scale, __uint_as_float(qr[4 * e + 1]) * p.scale,
+                                  __uint_as_float(qr[4 * e + 2]) * p.scale, __uint_as_float(qr[4 * e + 3]) * p.scale));
+        }
       }
     }
-  } else if (warp == 8) {
+  } else if (warp == 12) {
     // ======================= tensor-core issuer ==============================
     auto wwait = [&](int bi, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(bar(bi), parity, abort_flag));
@@ -498,7 +513,10 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
         const uint32_t o = (k * 16 * 128) >> 4;
-        if (elect_one()) mma_ts(tDV, tST + 8 * k, dO_mn + so + o, L::IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
+        // Pᵀ of queries [16k, 16k + 16): columns 8k.. for the first half, 32 + 8k..
+        // for the second (written over the Sᵀ columns that half's warps read)
+        const uint32_t pa = uint32_t(8 * k + (k >= 4 ? 32 : 0));
+        if (elect_one()) mma_ts(tDV, tST + pa, dO_mn + so + o, L::IDESC_KV, (n > 0 || k > 0) ? 1u : 0u);
       }
       if (next) {
         // Sᵀ of the next block over cols [0, 128): Pᵀ (cols [0, 64)) must have
@@ -535,7 +553,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       mbar_wait(bar(L::B_DONE), 0, nullptr);
     }
     __syncwarp();
-  } else if (warp == 9) {
+  } else if (warp == 13) {
     // ======================= TMA producer ====================================
     if (lane == 0 && total > 0) {
       tma_prefetch_desc(&tmQ);
@@ -572,7 +590,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     __syncwarp();
   }
 
-  if (warp == 10) {
+  if (warp == 14) {
     // ======================= lse / delta stager ==============================
     // lane l stages query rows l, l + 32, l + 64, l + 96 of each block once
     // every elementwise thread arrived on B_PB of the block before (its last
@@ -608,7 +626,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const volatile int* cnt = reinterpret_cast<const volatile int*>(smem + L::OFF_MISC);
     (void)(same_count(cnt[2], total) && same_count(cnt[3], total) && same_count(cnt[4], total));
   }
-  if (warp == 8) {
+  if (warp == 12) {
     tc_fence_after();
     tmem_dealloc(tmem, L::TMEM_COLS);
   }
