@@ -81,6 +81,11 @@ SHAPES = [
     ((1, 2, 2, 257, 257, 64), True, -1),       # d = 64
     ((1, 2, 2, 1024, 1024, 128), True, -1),    # many blocks per key block
     ((1, 2, 2, 160, 333, 64), False, 40),      # window without causal, d = 64
+    # mask edges inside one query half of a block only (each half of a block's
+    # queries is formed by its own elementwise warps)
+    ((1, 2, 2, 192, 192, 128), True, 100),
+    ((2, 4, 2, 320, 200, 64), True, 70),       # rows without keys, GQA, d = 64
+    ((1, 2, 2, 130, 450, 128), False, 90),     # window without causal, Nq < Nk
 ]
 
 
