@@ -212,8 +212,8 @@ struct BwdLayout {
   static constexpr int B_QDE = 3;    // Q_i, dO_i stage free again, + stage
   static constexpr int B_SS = 5;     // Sᵀ in TMEM
   static constexpr int B_SP = 6;     // dPᵀ in TMEM (and the previous dQ product done)
-  static constexpr int B_PA = 7;     // Pᵀ written (128 elementwise arrivals)
-  static constexpr int B_PB = 8;     // dSᵀ written to shared memory (128 arrivals)
+  static constexpr int B_PA = 7;     // Pᵀ written (256 elementwise arrivals)
+  static constexpr int B_PB = 8;     // dSᵀ written to shared memory (256 arrivals)
   static constexpr int B_DVD = 9;    // dV product of the block complete (issuer only)
   static constexpr int B_QR = 10;    // dQ_i in TMEM
   static constexpr int B_QF = 11;    // dQ_i read out (128 dQ-warp arrivals)
